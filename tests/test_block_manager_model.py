@@ -1,0 +1,127 @@
+"""Pins for the block-manager model (oracle/block_manager.py) against the pages' rules and
+worked examples."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle.block_manager import BlockManagerModel, OutOfBlocks
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_pages_waste_examples():
+    with open(os.path.join(GOLDEN, "waste_examples.json")) as f:
+        g = json.load(f)
+    for c in g["cases"]:
+        assert c["contiguous_reserved"] - c["tokens"] == c["contiguous_wasted"]
+        bm = BlockManagerModel(200, g["block_size"])
+        bm.add_seq("a", 0)
+        for _ in range(c["tokens"]):          # on-demand: one slot per generated token
+            bm.append_slot("a")
+        assert len(bm.block_table("a")) == c["paged_blocks"]
+        assert len(bm.block_table("a")) * g["block_size"] == c["paged_slots"]
+        assert bm.waste("a") == c["paged_wasted"]
+        assert bm.num_free() == 200 - c["paged_blocks"]
+
+
+def test_on_demand_allocation_only_at_block_boundaries():
+    bm = BlockManagerModel(10, 16, free_order=[3, 1, 4, 0, 5, 9, 2, 6, 8, 7])
+    bm.add_seq(0, 0)
+    slots = [bm.append_slot(0)[0] for _ in range(40)]
+    assert bm.block_table(0) == [3, 1, 4]
+    assert slots == [3 * 16 + i for i in range(16)] + [1 * 16 + i for i in range(16)] + \
+        [4 * 16 + i for i in range(8)]
+    assert bm.waste(0) == 8
+
+
+def test_fork_shares_blocks_and_copy_on_write_follows_refcount():
+    bm = BlockManagerModel(40, 16)
+    bm.add_seq("p", 20)                       # blocks 0, 1 (block 1 holds 4 tokens)
+    for c in range(1, 4):
+        bm.fork("p", c)
+    assert [bm.refcount(b) for b in (0, 1)] == [4, 4]
+    pairs = []
+    for s in ("p", 1, 2, 3):
+        slot, cow = bm.append_slot(s)
+        pairs.append(cow)
+    # the first three holders see refcount > 1 and copy; the last sees 1 and writes in place
+    assert pairs == [(1, 2), (1, 3), (1, 4), None]
+    assert bm.block_table("p") == [0, 2] and bm.block_table(3) == [0, 1]
+    assert [bm.refcount(b) for b in range(5)] == [4, 1, 1, 1, 1]
+    # appends that stay in a now-private block never copy again
+    for s in ("p", 1, 2, 3):
+        assert bm.append_slot(s)[1] is None
+
+
+def test_fork_at_block_boundary_needs_no_copy():
+    bm = BlockManagerModel(20, 16)
+    bm.add_seq(0, 32)
+    bm.fork(0, 1)
+    _, c0 = bm.append_slot(0)
+    _, c1 = bm.append_slot(1)
+    assert c0 is None and c1 is None and bm.block_table(0)[:2] == bm.block_table(1)[:2]
+
+
+def test_free_returns_blocks_fifo_when_refcount_reaches_zero():
+    bm = BlockManagerModel(6, 16)
+    bm.add_seq("a", 33)                       # 0, 1, 2
+    bm.fork("a", "b")
+    bm.free_seq("a")
+    assert bm.free_order() == [3, 4, 5]
+    bm.free_seq("b")
+    assert bm.free_order() == [3, 4, 5, 0, 1, 2]
+    assert all(bm.refcount(b) == 0 for b in range(6))
+
+
+def test_out_of_blocks_changes_nothing():
+    bm = BlockManagerModel(3, 16)
+    with pytest.raises(OutOfBlocks):
+        bm.add_seq(0, 64)
+    assert bm.num_free() == 3 and 0 not in bm.tables
+    bm.add_seq(0, 32)
+    bm.add_seq(1, 16)
+    state = (list(bm.free), list(bm.ref), {k: list(v) for k, v in bm.tables.items()},
+             dict(bm.lens))
+    with pytest.raises(OutOfBlocks):
+        bm.append_slots([0, 1])
+    assert state == (list(bm.free), list(bm.ref), {k: list(v) for k, v in bm.tables.items()},
+                     dict(bm.lens))
+
+
+def test_random_traffic_invariants():
+    rng = np.random.default_rng(7)
+    NB = 64
+    bm = BlockManagerModel(NB, 16, free_order=rng.permutation(NB))
+    live, nxt = [], 0
+    for step in range(3000):
+        op = rng.integers(0, 10)
+        try:
+            if op == 0 or not live:
+                bm.add_seq(nxt, int(rng.integers(0, 40)))
+                live.append(nxt)
+                nxt += 1
+            elif op == 1:
+                bm.fork(live[int(rng.integers(len(live)))], nxt)
+                live.append(nxt)
+                nxt += 1
+            elif op == 2:
+                s = live.pop(int(rng.integers(len(live))))
+                bm.free_seq(s)
+            else:
+                bm.append_slot(live[int(rng.integers(len(live)))])
+        except OutOfBlocks:
+            s = live.pop(0)
+            bm.free_seq(s)
+        # reference counts equal the number of table entries naming each block
+        count = [0] * NB
+        for s in live:
+            for b in bm.block_table(s):
+                count[b] += 1
+        assert count == bm.ref
+        # free blocks are exactly the unreferenced ones; nothing is lost or duplicated
+        assert sorted(bm.free_order()) == [b for b in range(NB) if count[b] == 0]
+        # only the last block of a sequence is partly empty
+        for s in live:
+            assert 0 <= bm.waste(s) < 16 or bm.seq_len(s) == 0
