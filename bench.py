@@ -1,0 +1,589 @@
+"""Benchmark of the paged decode path: KV GB/s, sequences/s and fraction of HBM roofline.
+
+One step = one pass of the whole hot path over one batch: copy-on-write block copies (when the
+workload forks), kv_write of each sequence's new token, and paged decode attention (with the
+split / log-sum-exp reduce for sequences longer than one partition).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload opt13b|gqa|long|fork]
+                    [--impl pkv|reference] [--no-cpu-baseline]
+
+N > 1 runs under torchrun, one process per GPU; every rank decodes its own replica of the
+batch (weak scaling, no data-path collective); time is the max over ranks.  Rank 0 prints
+one JSON line.  ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload on the host cores.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s & seqs/s, % of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_TEXT = {
+    "opt13b": "OPT-13B-shaped decode: 64 seqs, 40 heads MHA, head_dim 128, fp16 KV, block 16, "
+              "context lognormal(median 512, sigma 1) clipped 16..2048, shuffled placement, "
+              "pool 1.1x need, kv_write of one token per sequence",
+    "gqa": "GQA decode (Llama-3-8B-like): 128 seqs, 32 q / 8 kv heads, head_dim 128, bf16 KV, "
+           "block 16, context uniform 256..4096, shuffled placement, kv_write of one token per "
+           "sequence",
+    "long": "long-context split decode: 8 seqs x 32768 tokens, 32 q / 8 kv heads, head_dim 128, "
+            "bf16 KV, block 16, fully shuffled blocks, 512-token partitions + LSE reduce",
+    "fork": "parallel-sampling fork: 16 prompts x 8 samples sharing 1025 prefilled tokens, first "
+            "decode step (112 copy-on-write block copies, 128 kv_writes, decode over 1026 "
+            "tokens), fp16, 32 heads MHA, head_dim 128, block 16",
+}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="opt13b", choices=sorted(WORKLOAD_TEXT))
+    ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
+    ap.add_argument("--partition-tokens", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+# ---- workload construction ---------------------------------------------------------------
+def build_workload(name, model_block_manager=False):
+    """Return (Workload, cow_pairs int32 [P, 2]).  The fork workload's tables come from a
+    block manager: the product's C++ one, or the oracle's Python model for the CPU arm."""
+    from paged_kv_cache_392_b200 import workloads as W
+    if name != "fork":
+        return W.CONFIGS[name](), np.zeros((0, 2), np.int32)
+    f = W.FORK
+    NB = W.fork_pool_blocks()
+    rng = np.random.default_rng(f["seed"])
+    if model_block_manager:
+        from oracle.block_manager import BlockManagerModel
+        bm = _ModelAdapter(BlockManagerModel(NB, free_order=rng.permutation(NB)))
+    else:
+        from paged_kv_cache_392_b200 import binding as B
+        bm = B.BlockManager(NB, free_order=rng.permutation(NB))
+    seqs = []
+    prompt = f["prompt_tokens"] + f["shared_generated"]
+    for p in range(f["num_prompts"]):
+        bm.add_seq(p * f["samples"], prompt)
+        for k in range(1, f["samples"]):
+            bm.fork(p * f["samples"], p * f["samples"] + k)
+        seqs += [p * f["samples"] + k for k in range(f["samples"])]
+    slots, pairs = bm.append_slots(seqs)
+    maxB = -(-(prompt + f["steps"]) // 16)
+    bt, lens = bm.block_tables(seqs, maxB)
+    wl = W.Workload(name="fork", num_seqs=len(seqs), num_q_heads=f["num_heads"],
+                    num_kv_heads=f["num_heads"], head_dim=f["head_dim"], dtype=f["dtype"],
+                    context_lens=lens, block_tables=bt, num_blocks=NB,
+                    free_order=np.asarray(bm.free_order(), np.int32), slot_mapping=slots,
+                    scale=1.0 / math.sqrt(f["head_dim"]), seed=f["seed"])
+    wl.extra["unique_blocks"] = NB - bm.num_free()
+    bm.close()
+    return wl, pairs
+
+
+class _ModelAdapter:
+    """The oracle block-manager model behind the product manager's batch interface."""
+
+    def __init__(self, model):
+        self.m = model
+
+    def add_seq(self, s, n):
+        self.m.add_seq(s, n)
+
+    def fork(self, p, c):
+        self.m.fork(p, c)
+
+    def append_slots(self, seqs):
+        slots, pairs = self.m.append_slots(seqs)
+        return np.asarray(slots, np.int64), np.asarray(pairs, np.int32).reshape(-1, 2)
+
+    def block_tables(self, seqs, maxB):
+        bt = np.full((len(seqs), maxB), -1, np.int32)
+        for i, s in enumerate(seqs):
+            t = self.m.block_table(s)
+            bt[i, :len(t)] = t
+        return bt, np.array([self.m.seq_len(s) for s in seqs], np.int32)
+
+    def num_free(self):
+        return self.m.num_free()
+
+    def free_order(self):
+        return self.m.free_order()
+
+    def close(self):
+        pass
+
+
+def algorithmic_bytes(wl, pairs, split_rows=0, pmax_used=None):
+    """Bytes one step must move, counted from the definition of each kernel's work."""
+    es = wl.elem_size
+    S, Hq, Hkv, D = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
+    kv = wl.kv_bytes()                                    # K and V of every cached token
+    qo = S * Hq * D * es * 2                              # q read + out written
+    tables = int(((wl.context_lens + 15) // 16).sum()) * 4 + S * 4
+    ws = 0
+    if split_rows:                                        # partials written + read
+        ws = split_rows * (D + 2) * 4 * 2
+    write = S * Hkv * D * es * 2 * 2 + S * 8              # kv_write: read new + write pool
+    copy = len(pairs) * Hkv * 16 * D * es * 2 * 2         # each pair: read + write K and V
+    return {"kv": kv, "decode": kv + qo + tables + ws, "kv_write": write, "kv_copy": copy,
+            "step": kv + qo + tables + ws + write + copy}
+
+
+def split_rows(wl, partition_tokens):
+    """(query-head rows, partitions) of sequences that span more than one partition."""
+    pt = partition_tokens or 512
+    nparts = -(-wl.context_lens.astype(np.int64) // pt)
+    multi = nparts[nparts > 1]
+    return int(multi.sum()) * wl.num_q_heads, int(nparts.max())
+
+
+# ---- environment: peaks, clocks, profile traffic ----------------------------------------
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu summary for this workload, or
+    None when there is none or it was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "paged_attn_decode_%s.md" % workload)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not m or not sha or sha.group(1) != kernel_source_sha():
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background (every 100 ms)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index      # nvidia-smi -i argument (GPU UUID or index)
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if not self.proc:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- distributed plumbing -----------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend="nccl"):
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(dist, value, device):
+    """Max of a float over all ranks (identity with one rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---- the CUDA path --------------------------------------------------------------------------
+def gpu_uuid(torch, device):
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(device.index)
+
+
+def run_pkv(args):
+    import torch
+    from paged_kv_cache_392_b200 import binding as B
+    from paged_kv_cache_392_b200 import build as pbuild
+    from paged_kv_cache_392_b200 import workloads as W
+
+    world, rank, local = dist_env()
+    pbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world)
+
+    wl, pairs = build_workload(args.workload)
+    pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens
+    vals = W.make_values(wl, device)
+    q, kp, vp, kn, vn = (vals[k] for k in ("q", "k_pool", "v_pool", "k_new", "v_new"))
+    bt = torch.from_numpy(wl.block_tables).to(device)
+    lens = torch.from_numpy(wl.context_lens).to(device)
+    slots = torch.from_numpy(np.ascontiguousarray(wl.slot_mapping, np.int64)).to(device)
+    pairs_d = torch.from_numpy(np.ascontiguousarray(pairs, np.int32)).to(device)
+    out = torch.empty_like(q)
+    desc = B.decode_desc(q, kp, vp, bt, pt)
+    ws_bytes = B.attn_workspace_bytes(desc)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+    npairs = len(pairs)
+    rows_split, pmax = split_rows(wl, pt)
+    nbytes = algorithmic_bytes(wl, pairs, rows_split)
+
+    def step():
+        if npairs:
+            B.kv_copy_blocks(pairs_d, kp, vp)
+        B.kv_write(kn, vn, slots, kp, vp)
+        B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
+                            partition_tokens=pt)
+
+    launches_per_step = (1 if npairs else 0) + 1 + 1 + (1 if pmax > 1 else 0)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    faults = B.device_faults(clear=True)
+    if faults:
+        raise RuntimeError("device faults during warm-up: %s" % faults)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_uuid(torch, device))
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0.record()
+    for i in range(K):
+        if npairs:
+            B.kv_copy_blocks(pairs_d, kp, vp)
+        B.kv_write(kn, vn, slots, kp, vp)
+        ev[i][0].record()
+        B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
+                            partition_tokens=pt)
+        ev[i][1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    sampler.stop()
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(dist, ms_local, device)
+    decode_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    decode_ms = max_over_ranks(dist, decode_ms, device)
+    faults = B.device_faults(clear=True)
+    if faults:
+        raise RuntimeError("device faults during timing: %s" % faults)
+
+    # ---- end to end through the public API with host buffers -------------------------
+    pin = {k: v.cpu().pin_memory() for k, v in (("q", q), ("kn", kn), ("vn", vn),
+                                                 ("slots", slots), ("bt", bt),
+                                                 ("lens", lens), ("pairs", pairs_d))}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = out_h.numel() * out_h.element_size()
+    stream = torch.cuda.current_stream(device)
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        kn.copy_(pin["kn"], non_blocking=True)
+        vn.copy_(pin["vn"], non_blocking=True)
+        slots.copy_(pin["slots"], non_blocking=True)
+        bt.copy_(pin["bt"], non_blocking=True)
+        lens.copy_(pin["lens"], non_blocking=True)
+        if npairs:
+            pairs_d.copy_(pin["pairs"], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    Ke = max(1, min(K, 500))
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(Ke):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ke, device)
+    barrier(dist, device)
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        step_ms = ms / K
+        kv_gbs = world * nbytes["kv"] / (step_ms * 1e-3) / 1e9
+        achieved = nbytes["decode"] / (decode_ms * 1e-3) / 1e9
+        traffic = profile_traffic(args.workload)
+        result = {
+            "metric": METRIC,
+            "value": round(kv_gbs, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32 accumulate over %s KV" % wl.dtype,
+            "data": "synthetic (seeded), no weights",
+            "seqs_per_s": round(world * wl.num_seqs / (step_ms * 1e-3), 1),
+            "hbm_frac_step": round(kv_gbs / world / peak, 4),
+            "config": {
+                "workload": WORKLOAD_TEXT[args.workload],
+                "name": args.workload,
+                "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
+                "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                "block_size": 16, "kv_dtype": wl.dtype,
+                "context_tokens": int(wl.context_lens.sum()),
+                "partition_tokens": pt or 512, "cow_pairs_per_step": npairs,
+                "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
+                "l2": "no flush: KV working set %.2f GB per step > 126 MB L2" %
+                      (nbytes["kv"] / 1e9),
+                "parallelism": "replicas x%d" % world,
+            },
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "paged_attn_decode (decode + lse_reduce)",
+                "achieved": round(achieved, 1),
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+                "traffic": traffic,
+                "algorithmic_bytes": nbytes["decode"],
+                "avg_launch_ms": round(decode_ms, 5),
+            },
+            "e2e": {"value": round(world * nbytes["kv"] / (e2e_ms * 1e-3) / 1e9, 2),
+                    "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": Ke},
+            "gpu_launches": K * launches_per_step,
+            "clocks": sampler.summary(),
+        }
+        if wl.name == "fork":
+            uniq = wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim * \
+                wl.elem_size * 2
+            result["config"]["unique_kv_bytes"] = uniq
+            result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(wl, vals, args.cpu_seconds)
+    if dist is not None:
+        barrier(dist, device)
+        dist.destroy_process_group()
+    return result
+
+
+# ---- the fp64 oracle on the host cores ------------------------------------------------------
+def _seq_kv_bytes(wl, s):
+    return int(wl.context_lens[s]) * wl.num_kv_heads * wl.head_dim * wl.elem_size * 2
+
+
+def _pick_sequences(wl, bytes_budget):
+    """Sequences, in a seeded shuffled order, until their KV bytes reach the budget."""
+    order = np.random.default_rng(12345).permutation(wl.num_seqs)
+    chosen, total = [], 0
+    for s in order:
+        chosen.append(int(s))
+        total += _seq_kv_bytes(wl, s)
+        if total >= bytes_budget:
+            break
+    return sorted(chosen), total
+
+
+def _oracle_rows(wl, seqs):
+    return np.array([(s, h) for s in seqs for h in range(wl.num_q_heads)], np.int32)
+
+
+def _calibrate(oracle, wl, host):
+    """Oracle KV bytes per second on this host, from one mid-sized sequence."""
+    s = int(np.argsort(wl.context_lens)[wl.num_seqs // 2])
+    rows = _oracle_rows(wl, [s])
+    t = time.perf_counter()
+    oracle.paged_attn_decode(host["q"], host["k_pool"], host["v_pool"], wl.block_tables,
+                             wl.context_lens, wl.scale, wl.dtype, rows=rows)
+    dt = max(time.perf_counter() - t, 1e-4)
+    return _seq_kv_bytes(wl, s) / dt
+
+
+def cpu_baseline(wl, vals, seconds):
+    import oracle
+    from paged_kv_cache_392_b200 import workloads as W
+    host = {k: W.to_numpy_bits(vals[k]) for k in ("q", "k_pool", "v_pool")}
+    rate = _calibrate(oracle, wl, host)
+    seqs, nbytes = _pick_sequences(wl, rate * seconds)
+    rows = _oracle_rows(wl, seqs)
+    t = time.perf_counter()
+    oracle.paged_attn_decode(host["q"], host["k_pool"], host["v_pool"], wl.block_tables,
+                             wl.context_lens, wl.scale, wl.dtype, rows=rows)
+    dt = time.perf_counter() - t
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "seqs_per_s": round(len(seqs) / dt, 3), "seconds": round(dt, 2),
+            "sample": "decode attention of %d of %d sequences (all %d query heads, %d context "
+                      "tokens) of the same batch, fp64, exact two-pass softmax" %
+                      (len(seqs), wl.num_seqs, wl.num_q_heads,
+                       int(wl.context_lens[seqs].sum()))}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    import torch
+    from paged_kv_cache_392_b200 import workloads as W
+    wl, pairs = build_workload(args.workload, model_block_manager=True)
+    vals = W.make_values(wl, "cpu", torch=torch)
+    host = {k: W.to_numpy_bits(v).copy() for k, v in vals.items()}
+    rate = _calibrate(oracle, wl, host)
+    budget_s = max(0.02, min(1.0, 90.0 / max(1, args.steps + args.warmup)))
+    seqs, nbytes = _pick_sequences(wl, rate * budget_s)
+    rows = _oracle_rows(wl, seqs)
+    sel = np.array(seqs)
+    chosen = set(seqs)
+    # the sample's copy-on-write pairs: those whose destination one of its sequences maps
+    dst_of = {int(b) for s in seqs for b in wl.block_tables[s] if b >= 0}
+    sp = np.array([p for p in pairs if int(p[1]) in dst_of], np.int32).reshape(-1, 2)
+    kn, vn = host["k_new"][sel].copy(), host["v_new"][sel].copy()
+    slots = wl.slot_mapping[sel].copy()
+
+    def step():
+        if len(sp):
+            oracle.kv_copy_blocks(sp, host["k_pool"], host["v_pool"])
+        oracle.kv_write(kn, vn, slots, host["k_pool"], host["v_pool"])
+        oracle.paged_attn_decode(host["q"], host["k_pool"], host["v_pool"], wl.block_tables,
+                                 wl.context_lens, wl.scale, wl.dtype, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t) / max(1, args.steps)
+    gbs = nbytes / dt / 1e9
+    sample = ("per step: kv_write + decode attention of %d of %d sequences (%d context "
+              "tokens, all %d query heads)%s, fp64 oracle" %
+              (len(seqs), wl.num_seqs, int(wl.context_lens[sel].sum()), wl.num_q_heads,
+               (", %d copy-on-write pairs" % len(sp)) if len(sp) else ""))
+    assert len(chosen) == len(seqs)
+    return {
+        "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded), no weights", "impl": "reference",
+        "seqs_per_s": round(len(seqs) / dt, 3),
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
+                   "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+                   "block_size": 16, "kv_dtype": wl.dtype},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "kind": "oracle",
+                         "cores": oracle.num_threads(), "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, _ = dist_env()
+    if args.gpus != world and world > 1:
+        print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
+    res = run_reference(args) if args.impl == "reference" else run_pkv(args)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * pkv.h -- C ABI of libpkv, the B200 (sm_100a) paged KV-cache decode path.
+ *
+ * The operations follow the PagedAttention description in "Memory Optimization in LLM
+ * Serving with PagedAttention" (sections "How PagedAttention Works" and "Advanced
+ * Capabilities: Memory Sharing with Copy-on-Write") and "vLLM and PagedAttention: How Ideas
+ * from Operating Systems Accelerated LLM Inference": the KV cache is a pool of fixed-size
+ * physical blocks of 16 tokens, each sequence reaches its tokens through a block table, a
+ * custom kernel gathers the scattered blocks to compute attention, and shared blocks are
+ * copied before a sequence writes into them.
+ *
+ * Conventions (every function):
+ *   - Returns pkv_status; PKV_OK is 0.  On failure pkv_last_error() (per calling thread)
+ *     describes the first problem found.  Nothing is launched when host-side validation fails.
+ *   - Tensor pointers are DEVICE pointers owned by the caller unless a parameter says "host".
+ *     The library allocates no device memory on these paths; scratch space is passed in.
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default stream).  Launches
+ *     are asynchronous; the calls return once the kernels are queued.
+ *   - dtype is one of pkv_dtype; q, out, the pools and the new K/V all use the same dtype.
+ *   - Pool layout: k_pool and v_pool are row-major [num_blocks][num_kv_heads][block_size]
+ *     [head_dim], so one (block, kv head) is a contiguous block_size*head_dim run.
+ *     Token t of sequence s is at block block_tables[s*max_blocks_per_seq + t/16], offset
+ *     t%16.  A slot number names (block, offset) as block*16 + offset.
+ *   - Device-side checks: values only the GPU sees (context lengths, table entries, slots,
+ *     block ids) are range-checked by the kernels before any access.  A bad value is skipped
+ *     (never dereferenced) and sets a bit in the device fault word that
+ *     pkv_device_faults() reads.  Outputs that depended on a bad value are unspecified.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID = 1,      /* bad argument (null pointer, shape, alignment, range)   */
+    PKV_ERR_OOM = 2,          /* block manager: not enough free blocks; state unchanged */
+    PKV_ERR_UNSUPPORTED = 3,  /* valid but not built: head_dim, dtype, block size       */
+    PKV_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed                   */
+    PKV_ERR_NOT_FOUND = 5     /* block manager: unknown sequence id                     */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+
+/* Bits of the device fault word. */
+#define PKV_FAULT_BAD_LEN   0x1u  /* context_lens[s] outside [1, max_blocks_per_seq*16]  */
+#define PKV_FAULT_BAD_BLOCK 0x2u  /* block table entry outside [0, num_blocks)          */
+#define PKV_FAULT_BAD_SLOT  0x4u  /* slot outside [0, num_blocks*16) and not -1         */
+#define PKV_FAULT_BAD_PAIR  0x8u  /* copy pair naming a block outside [0, num_blocks)   */
+#define PKV_FAULT_TIMEOUT   0x10u /* a bounded wait on a shared-memory barrier gave up  */
+
+/* Shape of one decode batch and of the pools it reads. */
+typedef struct pkv_attn_desc {
+    int32_t num_seqs;            /* S                                                   */
+    int32_t num_q_heads;         /* H_q                                                 */
+    int32_t num_kv_heads;        /* H_kv; H_q % H_kv == 0, query head h reads kv head   */
+                                 /* h / (H_q / H_kv)                                    */
+    int32_t head_dim;            /* D: 64 or 128                                        */
+    int32_t block_size;          /* tokens per block: 16                                */
+    int32_t num_blocks;          /* NB, physical blocks in each pool                    */
+    int32_t max_blocks_per_seq;  /* row stride of block_tables                          */
+    int32_t dtype;               /* pkv_dtype                                           */
+    int32_t partition_tokens;    /* context split for long sequences: 0 = library's     */
+                                 /* choice, else a multiple of 16                       */
+} pkv_attn_desc;
+
+/* Last error message of the calling thread ("" if none).  Never NULL. */
+const char *pkv_last_error(void);
+
+/* Library version string. */
+const char *pkv_version(void);
+
+/*
+ * Scratch bytes paged_attn_decode needs for split-context partial results (0 when no
+ * sequence of this shape can span more than one partition).  Depends only on the
+ * descriptor.  Returns 0 and sets the last error on an invalid descriptor.
+ */
+size_t pkv_attn_workspace_bytes(const pkv_attn_desc *desc);
+
+/*
+ * Single-token decode attention over the paged KV cache ("Memory Optimization in LLM Serving
+ * with PagedAttention", section "How PagedAttention Works": the kernel gathers the scattered
+ * KV blocks through the block table to compute attention).  For every sequence s and query
+ * head h, with L = context_lens[s] and kv head hk = h / (H_q / H_kv):
+ *     x_t = scale * <q[s,h,:], K_t>   for t in [0, L), K_t read through the block table
+ *     out[s,h,:] = sum_t softmax(x)_t * V_t
+ * accumulated in fp32 and rounded once to dtype.
+ *   q            [S, H_q, D] dtype
+ *   k_pool/v_pool [NB, H_kv, 16, D] dtype, 16-byte aligned
+ *   block_tables [S, max_blocks_per_seq] int32; only the first ceil(L/16) entries of a row
+ *                are read
+ *   context_lens [S] int32, each in [1, max_blocks_per_seq*16] (checked on the device)
+ *   out          [S, H_q, D] dtype
+ *   workspace    at least pkv_attn_workspace_bytes(desc) bytes, 256-byte aligned (may be
+ *                NULL when that is 0); overwritten; calls that share it must not overlap
+ * Sequences longer than the partition size are split; each partition is computed
+ * independently and a second kernel merges the partitions by log-sum-exp.
+ */
+pkv_status paged_attn_decode(const pkv_attn_desc *desc, const void *q, const void *k_pool,
+                             const void *v_pool, const int32_t *block_tables,
+                             const int32_t *context_lens, float scale, void *out,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Scatter each new token's K and V into its slot ("Memory Optimization in LLM Serving with
+ * PagedAttention", section "How PagedAttention Works": blocks are filled on demand as
+ * generation proceeds).  For token t and kv head h:
+ *     k_pool[slot/16, h, slot%16, :] = k_new[t, h, :]   (and the same for V)
+ * bytes copied unchanged.  slot_mapping[t] == -1 skips token t.
+ *   k_new/v_new  [num_tokens, H_kv, D] dtype
+ *   slot_mapping [num_tokens] int64, distinct values in [0, NB*16) or -1
+ * Only num_kv_heads, head_dim, block_size, num_blocks and dtype of desc are used.
+ */
+pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
+                    const int64_t *slot_mapping, int32_t num_tokens, void *k_pool,
+                    void *v_pool, void *stream);
+
+/*
+ * Copy-on-write block copy ("Memory Optimization in LLM Serving with PagedAttention",
+ * section "Advanced Capabilities: Memory Sharing with Copy-on-Write": before a sequence
+ * writes into a block it shares, the block's content is copied to a fresh block).  For each
+ * pair i, physical block src_dst_pairs[2i+1] of both pools (every kv head and slot) becomes a
+ * byte copy of block src_dst_pairs[2i].
+ *   src_dst_pairs [num_pairs][2] int32, device memory; destinations distinct and never a
+ *                 source of another pair (otherwise the result is unspecified but in bounds)
+ * Only num_kv_heads, head_dim, block_size, num_blocks and dtype of desc are used.
+ */
+pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pairs,
+                          int32_t num_pairs, void *k_pool, void *v_pool, void *stream);
+
+/*
+ * Read the device fault word of the current device into *faults (host) after the work
+ * queued on stream so far has finished; clear != 0 resets it to 0.  Synchronises stream.
+ */
+pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Host block manager ("Memory Optimization in LLM Serving with PagedAttention", sections
+ * "How PagedAttention Works" (on-demand allocation, fragmentation only in the last block)
+ * and "Advanced Capabilities: Memory Sharing with Copy-on-Write" (shared blocks, reference
+ * counts, copy before write); "vLLM and PagedAttention: How Ideas from Operating Systems
+ * Accelerated LLM Inference" (16-token blocks, fork-style sharing for parallel sampling)).
+ *
+ * Host only: it hands out block ids and slots and never touches device memory.  Sequence
+ * ids are caller-chosen int64.  The free list is first-in first-out (allocation takes its
+ * head, a block whose reference count drops to 0 joins its tail).  A call that fails with
+ * PKV_ERR_OOM changes nothing.  Not thread-safe: one thread per manager at a time.
+ * ------------------------------------------------------------------------------------- */
+typedef struct pkv_bm pkv_bm;
+
+/* initial_free_order: host [num_blocks] permutation of 0..num_blocks-1, or NULL for
+ * ascending order.  block_size must be 16. */
+pkv_status pkv_bm_create(int32_t num_blocks, int32_t block_size,
+                         const int32_t *initial_free_order, pkv_bm **out);
+void pkv_bm_destroy(pkv_bm *bm);
+
+/* Register sequence seq holding num_tokens tokens (a prompt): ceil(num_tokens/16) fresh
+ * blocks, all or nothing. */
+pkv_status pkv_bm_add_seq(pkv_bm *bm, int64_t seq, int32_t num_tokens);
+
+/* Give the next token of seq a slot.  If the token opens a new block, a fresh block is
+ * appended.  Otherwise, if the last block is shared (reference count > 1), a fresh block dst
+ * replaces it in seq's table, the old block's count drops by one, and (*cow_src, *cow_dst)
+ * = (old, dst) tells the caller to run kv_copy_blocks before writing; else both are -1. */
+pkv_status pkv_bm_append_slot(pkv_bm *bm, int64_t seq, int64_t *slot_out, int32_t *cow_src,
+                              int32_t *cow_dst);
+
+/* append_slot for n sequences in order, all or nothing.  slots_out [n] int64 (host);
+ * cow_pairs_out [n][2] int32 (host) receives *num_cow pairs. */
+pkv_status pkv_bm_append_slots(pkv_bm *bm, const int64_t *seqs, int32_t n,
+                               int64_t *slots_out, int32_t *cow_pairs_out,
+                               int32_t *num_cow);
+
+/* child maps the same physical blocks as parent (every count + 1) and has its length. */
+pkv_status pkv_bm_fork(pkv_bm *bm, int64_t parent, int64_t child);
+
+/* Drop seq; blocks whose count reaches 0 return to the free list in table order. */
+pkv_status pkv_bm_free_seq(pkv_bm *bm, int64_t seq);
+
+/* Copy seq's block table into out (host, capacity cap); *n = its length (also when
+ * cap < *n, in which case PKV_ERR_INVALID is returned and out holds the first cap). */
+pkv_status pkv_bm_block_table(const pkv_bm *bm, int64_t seq, int32_t *out, int32_t cap,
+                              int32_t *n);
+
+/* Pack the tables of n sequences into out [n][max_blocks] (host, -1 padded) and their
+ * lengths into lens_out [n] (host). */
+pkv_status pkv_bm_block_tables(const pkv_bm *bm, const int64_t *seqs, int32_t n,
+                               int32_t max_blocks, int32_t *out, int32_t *lens_out);
+
+pkv_status pkv_bm_seq_len(const pkv_bm *bm, int64_t seq, int32_t *len);
+pkv_status pkv_bm_refcount(const pkv_bm *bm, int32_t block, int32_t *count);
+int32_t pkv_bm_num_free(const pkv_bm *bm);
+int32_t pkv_bm_num_seqs(const pkv_bm *bm);
+
+/* Copy the free list, head first, into out (host, capacity cap); returns its length. */
+int32_t pkv_bm_free_list(const pkv_bm *bm, int32_t *out, int32_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

@@ -1,0 +1,477 @@
+// Paged decode attention for sm_100a.
+//
+// What it computes ("Memory Optimization in LLM Serving with PagedAttention", section "How
+// PagedAttention Works": a custom kernel gathers the scattered KV blocks through the block
+// table to compute attention): for each sequence s and query head h, softmax(q K^T * scale) V
+// over the sequence's context_lens[s] cached tokens, K/V rows fetched from the physical block
+// block_tables[s][t / 16], offset t % 16.
+//
+// How (B200 design):
+//   * one CTA per work unit (sequence, kv head, context partition); the CTA serves all
+//     H_q/H_kv query heads that share the kv head, so each K/V block is read from HBM once;
+//   * W consumer warps; warp w takes the unit's blocks w, w+W, w+2W, ...; each warp owns a
+//     ring of NSW shared-memory stages and keeps it full with the bulk async copy engine
+//     (one elected lane issues two contiguous 16*D-element copies, K and V, per block,
+//     completion counted in bytes on the stage's mbarrier, bounded waits);
+//   * per 16-token block: lane (c, r) owns 16-byte chunk c of the head dimension and tokens
+//     r, r+TPP, ...; it forms partial q.k sums from conflict-free 16-byte shared loads, a
+//     shuffle reduce-scatter finishes the dot products, then an online softmax (running
+//     max / sum, fp32, base-2 exponent with scale*log2(e) folded into q) and the P.V update;
+//   * at the end the W warps' (max, sum, unnormalised output) states are merged in shared
+//     memory; a unit covering the whole sequence writes the normalised output, otherwise it
+//     writes its partial state for the log-sum-exp reduce kernel below.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "faults.cuh"
+#include "ptx.cuh"
+
+namespace pkv {
+
+constexpr int kBlock = 16;                       // tokens per KV block
+constexpr uint64_t kWaitTimeoutNs = 1000000000;  // bounded shared-memory barrier waits (1 s)
+
+
+struct DecodeParams {
+    const void *q;
+    const void *k_pool;
+    const void *v_pool;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    void *out;
+    float *ws_o;   // [S][H_q][pmax][D] unnormalised partition outputs (split only)
+    float *ws_ml;  // [S][H_q][pmax][2]  partition (max, sum), base-2 units (split only)
+    int32_t S, Hq, Hkv, NB, maxB;
+    int32_t part_blocks;  // blocks per partition
+    int32_t pmax;         // partitions of the longest admissible sequence
+    float scale_log2;     // scale * log2(e)
+};
+
+// ---- element conversions --------------------------------------------------------------
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<float> {
+    static constexpr int kPer16B = 4;
+    __device__ static __forceinline__ void load(const uint4 &v, float (&f)[4]) {
+        f[0] = __uint_as_float(v.x);
+        f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z);
+        f[3] = __uint_as_float(v.w);
+    }
+    __device__ static __forceinline__ float from_float(float x) { return x; }
+};
+
+template <>
+struct Elem<__half> {
+    static constexpr int kPer16B = 8;
+    __device__ static __forceinline__ void load(const uint4 &v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+            float2 a = __half22float2(h);
+            f[2 * i] = a.x;
+            f[2 * i + 1] = a.y;
+        }
+    }
+    __device__ static __forceinline__ __half from_float(float x) { return __float2half_rn(x); }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int kPer16B = 8;
+    // bfloat16 is the upper half of a binary32: widening is a shift / mask.
+    __device__ static __forceinline__ void load(const uint4 &v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+    __device__ static __forceinline__ __nv_bfloat16 from_float(float x) {
+        return __float2bfloat16_rn(x);
+    }
+};
+
+// Store E floats as E elements of T (16 bytes for 16-bit T, 16 bytes for float).
+template <typename T, int E>
+__device__ __forceinline__ void store_row(T *dst, const float (&x)[E]) {
+    static_assert(E * sizeof(T) == 16, "one 16-byte vector");
+    union {
+        uint4 v;
+        T e[E];
+    } u;
+#pragma unroll
+    for (int i = 0; i < E; ++i) u.e[i] = Elem<T>::from_float(x[i]);
+    *reinterpret_cast<uint4 *>(dst) = u.v;
+}
+
+template <typename T, int D, int G, int W, int NSW>
+struct DecodeCfg {
+    static constexpr int ES = sizeof(T);
+    static constexpr int E = 16 / ES;             // elements per 16-byte chunk
+    static constexpr int CPR = D * ES / 16;       // chunks per token row
+    static constexpr int TPP = 32 / CPR;          // tokens per pass of the warp
+    static constexpr int NPASS = kBlock / TPP;    // passes per block
+    static constexpr int NV = NPASS * G;          // partial scores per lane
+    static constexpr int HG = G >= 2 ? G / 2 : 1; // heads per lane after the reduction
+    static constexpr int NE = G >= 2 ? G / 2 : 1; // softmax entries per lane
+    static constexpr int CHUNK = kBlock * D * ES; // bytes of one (block, kv head)
+    static constexpr int RING = W * NSW * 2 * CHUNK;
+    static constexpr int BARS = W * NSW * 8;
+    static constexpr int SCR = W * (kBlock * G + G) * 4;   // per-warp scores / rescale
+    static constexpr int MRG = W * G * (D + 2) * 4;        // cross-warp merge
+    static constexpr int SMEM = RING + BARS + SCR + MRG;
+    static_assert(CPR >= 8 && CPR <= 32, "head_dim * elem_size must be 128..512 bytes");
+    static_assert(NV <= 64, "too many partial scores per lane");
+};
+
+template <typename T, int D, int G, int W, int NSW>
+__global__ void __launch_bounds__(W * 32)
+paged_attn_decode_kernel(const DecodeParams p) {
+    using C = DecodeCfg<T, D, G, W, NSW>;
+    constexpr int E = C::E, CPR = C::CPR, TPP = C::TPP, NPASS = C::NPASS, NV = C::NV;
+    constexpr int HG = C::HG, NE = C::NE, CHUNK = C::CHUNK;
+    constexpr unsigned FULL = 0xffffffffu;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    pdl_launch_dependents();
+
+    const int bid = blockIdx.x;
+    const int part = bid % p.pmax;
+    const int rest = bid / p.pmax;
+    const int hk = rest % p.Hkv;
+    const int s = rest / p.Hkv;
+
+    const int L = p.context_lens[s];
+    if (L < 1 || L > p.maxB * kBlock) {
+        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, 0x1u);
+        return;
+    }
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
+    if (part >= nparts) return;
+    const int j0 = part * p.part_blocks;
+    const int nb = min(nblk, j0 + p.part_blocks) - j0;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int c = lane % CPR;   // 16-byte chunk of the head dimension
+    const int r = lane / CPR;   // token phase within a pass
+    const int nbw = nb > warp ? (nb - warp + W - 1) / W : 0;
+
+    unsigned char *ring = smem + warp * NSW * 2 * CHUNK;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::RING) + warp * NSW;
+    float *sc = reinterpret_cast<float *>(smem + C::RING + C::BARS) + warp * (kBlock * G + G);
+    float *al = sc + kBlock * G;
+    float *mo = reinterpret_cast<float *>(smem + C::RING + C::BARS + C::SCR);  // [W][G][D]
+    float *mml = mo + W * G * D;                                               // [W][G][2]
+
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < NSW; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const char *kbase = static_cast<const char *>(p.k_pool);
+    const char *vbase = static_cast<const char *>(p.v_pool);
+    const uint64_t policy = l2_evict_first_policy();
+
+    // Block-table entries of this warp's blocks, 32 at a time (lane i holds block i).
+    int tab_chunk = 0;
+    int32_t tab = lane < nbw ? btrow[(size_t)W * lane] : 0;
+
+    // Issue block i of this warp into stage i % NSW (all lanes call; lane 0 issues).
+    auto issue = [&](int i) {
+        if ((i >> 5) != tab_chunk) {
+            tab_chunk = i >> 5;
+            const int li = (tab_chunk << 5) + lane;
+            tab = li < nbw ? btrow[(size_t)W * li] : 0;
+        }
+        const int32_t phys = __shfl_sync(FULL, tab, i & 31);
+        if (lane == 0) {
+            uint64_t *bar = &bars[i % NSW];
+            unsigned char *dst = ring + (i % NSW) * 2 * CHUNK;
+            if ((unsigned)phys < (unsigned)p.NB) {
+                const size_t off = ((size_t)phys * p.Hkv + hk) * (size_t)CHUNK;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(bar, 2 * CHUNK);
+                bulk_g2s(dst, kbase + off, CHUNK, bar, policy);
+                bulk_g2s(dst + CHUNK, vbase + off, CHUNK, bar, policy);
+            } else {
+                atomicOr(&g_faults, 0x2u);
+                mbar_arrive(bar);  // complete the phase without data
+            }
+        }
+    };
+
+    const int npro = nbw < NSW ? nbw : NSW;
+    for (int i = 0; i < npro; ++i) issue(i);
+    int issued = npro;
+
+    // Query rows of the group, pre-scaled into base-2 logits.
+    float q[G][E];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+        const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + hh) * D;
+        const uint4 v = *reinterpret_cast<const uint4 *>(qrow + c * E);
+        Elem<T>::load(v, q[hh]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) q[hh][e] *= p.scale_log2;
+    }
+
+    float o[G][E];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[hh][e] = 0.f;
+    float m_run[NE], l_run[NE];
+#pragma unroll
+    for (int k = 0; k < NE; ++k) {
+        m_run[k] = -INFINITY;
+        l_run[k] = 0.f;
+    }
+
+    bool dead = false;
+    int i = 0;
+    for (; i < nbw; ++i) {
+        const int st = i % NSW;
+        if (!mbar_wait_bounded(&bars[st], (uint32_t)(i / NSW) & 1u, kWaitTimeoutNs)) {
+            if (lane == 0) atomicOr(&g_faults, 0x10u);
+            dead = true;
+            break;
+        }
+        const unsigned char *Ks = ring + st * 2 * CHUNK;
+        const unsigned char *Vs = Ks + CHUNK;
+        const int jb = j0 + warp + W * i;                // logical block
+        const int nvalid = min(kBlock, L - jb * kBlock); // tokens of this block in context
+
+        // ---- partial scores: v[ii * G + hh] over this lane's chunk -------------------
+        float v[NV];
+#pragma unroll
+        for (int ii = 0; ii < NPASS; ++ii) {
+            const int t = r + TPP * ii;
+            const uint4 kv = *reinterpret_cast<const uint4 *>(Ks + (t * CPR + c) * 16);
+            float kf[E];
+            Elem<T>::load(kv, kf);
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) a = fmaf(q[hh][e], kf[e], a);
+                v[ii * G + hh] = a;
+            }
+        }
+        // ---- reduce-scatter over the CPR lanes sharing a token phase ----------------
+        int n = NV;
+#pragma unroll
+        for (int m = CPR / 2; m >= 1; m >>= 1) {
+            if (n > 1) {
+                const bool up = (lane & m) != 0;
+                const int half = n / 2;
+#pragma unroll
+                for (int j = 0; j < NV / 2; ++j) {
+                    if (j < half) {
+                        const float send = up ? v[j] : v[j + half];
+                        const float keep = up ? v[j + half] : v[j];
+                        v[j] = keep + __shfl_xor_sync(FULL, send, m);
+                    }
+                }
+                n = half;
+            } else {
+                v[0] += __shfl_xor_sync(FULL, v[0], m);
+            }
+        }
+        // lane now holds the logits of token tt for heads hh0 .. hh0+HG-1
+        {
+            const int tt = r + TPP * (c >> 1);
+            const int hh0 = G >= 2 ? (c & 1) * HG : 0;
+#pragma unroll
+            for (int k = 0; k < HG; ++k) sc[tt * G + hh0 + k] = tt < nvalid ? v[k] : -INFINITY;
+        }
+        __syncwarp();
+
+        // ---- online softmax over the block: entry (head hh, token lane % 16) --------
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+            const int hh = G >= 2 ? (lane >> 4) + 2 * k : 0;
+            const int tt = lane & 15;
+            const float x = sc[tt * G + hh];
+            float bm = x;
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, m));
+            const float mn = fmaxf(m_run[k], bm);
+            const float pv = exp2f(x - mn);
+            float sum = pv;
+#pragma unroll
+            for (int m = 1; m < 16; m <<= 1) sum += __shfl_xor_sync(FULL, sum, m);
+            const float a = exp2f(m_run[k] - mn);
+            l_run[k] = l_run[k] * a + sum;
+            m_run[k] = mn;
+            sc[tt * G + hh] = pv;
+            if (tt == 0) al[hh] = a;
+        }
+        __syncwarp();
+
+        // ---- P.V ----------------------------------------------------------------------
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+            const float a = al[hh];
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[hh][e] *= a;
+        }
+#pragma unroll
+        for (int ii = 0; ii < NPASS; ++ii) {
+            const int t = r + TPP * ii;
+            if (t < nvalid) {
+                const uint4 vv = *reinterpret_cast<const uint4 *>(Vs + (t * CPR + c) * 16);
+                float vf[E];
+                Elem<T>::load(vv, vf);
+#pragma unroll
+                for (int hh = 0; hh < G; ++hh) {
+                    const float pr = sc[t * G + hh];
+#pragma unroll
+                    for (int e = 0; e < E; ++e) o[hh][e] = fmaf(pr, vf[e], o[hh][e]);
+                }
+            }
+        }
+        __syncwarp();
+
+        if (issued < nbw) {
+            issue(issued);
+            ++issued;
+        }
+    }
+    if (dead) {
+        // Let copies still in flight (blocks i .. issued-1, at most one per stage) land
+        // before the CTA retires; bounded as well.
+        for (int b = i; b < issued; ++b) {
+            (void)mbar_wait_bounded(&bars[b % NSW], (uint32_t)(b / NSW) & 1u, kWaitTimeoutNs);
+        }
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+            m_run[k] = -INFINITY;
+            l_run[k] = 0.f;
+        }
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[hh][e] = 0.f;
+    }
+
+    // ---- warp state -> shared memory ---------------------------------------------------
+#pragma unroll
+    for (int m = CPR; m < 32; m <<= 1)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[hh][e] += __shfl_xor_sync(FULL, o[hh][e], m);
+    if (lane < CPR) {
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+            for (int e = 0; e < E; ++e) mo[(warp * G + hh) * D + c * E + e] = o[hh][e];
+    }
+    if ((lane & 15) == 0) {
+#pragma unroll
+        for (int k = 0; k < NE; ++k) {
+            const int hh = G >= 2 ? (lane >> 4) + 2 * k : 0;
+            mml[(warp * G + hh) * 2 + 0] = m_run[k];
+            mml[(warp * G + hh) * 2 + 1] = l_run[k];
+        }
+    }
+    __syncthreads();
+
+    // ---- merge the W warps; write output or this partition's partial state -------------
+    constexpr int VPH = D / E;  // 16-byte output vectors per head
+    for (int idx = threadIdx.x; idx < G * VPH; idx += W * 32) {
+        const int hh = idx / VPH;
+        const int d0 = (idx % VPH) * E;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < W; ++w) M = fmaxf(M, mml[(w * G + hh) * 2]);
+        float den = 0.f, num[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) num[e] = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const float mw = mml[(w * G + hh) * 2];
+            const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            den += a * mml[(w * G + hh) * 2 + 1];
+#pragma unroll
+            for (int e = 0; e < E; ++e) num[e] += a * mo[(w * G + hh) * D + d0 + e];
+        }
+        const int h = hk * G + hh;
+        if (nparts == 1) {
+            const float inv = 1.f / den;
+#pragma unroll
+            for (int e = 0; e < E; ++e) num[e] *= inv;
+            store_row<T, E>(static_cast<T *>(p.out) + ((size_t)s * p.Hq + h) * D + d0, num);
+        } else {
+            const size_t row = ((size_t)s * p.Hq + h) * p.pmax + part;
+            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D + d0);
+#pragma unroll
+            for (int e = 0; e < E; e += 4)
+                dst[e / 4] = make_float4(num[e], num[e + 1], num[e + 2], num[e + 3]);
+            if (d0 == 0) {
+                p.ws_ml[row * 2] = M;
+                p.ws_ml[row * 2 + 1] = den;
+            }
+        }
+    }
+}
+
+// ---- log-sum-exp merge of the partitions of split sequences ----------------------------
+// out[s,h,:] = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p  (base-2 units,
+// which is the natural-log formula with every logit scaled by log2(e)).  One warp per row;
+// rows whose sequence fits in one partition were already written by the decode kernel.
+template <typename T, int D>
+__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams p) {
+    constexpr int DPL = D / 32;  // elements per lane
+    pdl_wait_primary();
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= p.S * p.Hq) return;
+    const int s = row / p.Hq;
+    const int L = p.context_lens[s];
+    if (L < 1 || L > p.maxB * kBlock) return;
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int np = (nblk + p.part_blocks - 1) / p.part_blocks;
+    if (np <= 1) return;
+    const float *ml = p.ws_ml + (size_t)row * p.pmax * 2;
+    const float *ob = p.ws_o + (size_t)row * p.pmax * D;
+
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, ml[2 * i]);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
+    float den = 0.f;
+    for (int i = lane; i < np; i += 32) den += exp2f(ml[2 * i] - M) * ml[2 * i + 1];
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+
+    float acc[DPL];
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
+    for (int i = 0; i < np; ++i) {
+        const float w = exp2f(ml[2 * i] - M);
+        const float *src = ob + (size_t)i * D + lane * DPL;
+#pragma unroll
+        for (int k = 0; k < DPL; ++k) acc[k] = fmaf(w, src[k], acc[k]);
+    }
+    const float inv = 1.f / den;
+    T *dst = static_cast<T *>(p.out) + (size_t)row * D + lane * DPL;
+#pragma unroll
+    for (int k = 0; k < DPL; ++k) dst[k] = Elem<T>::from_float(acc[k] * inv);
+}
+
+}  // namespace pkv

@@ -1,0 +1,293 @@
+// Host side of libpkv's CUDA path: argument validation, kernel selection and launches for
+// paged_attn_decode, kv_write and kv_copy_blocks, plus the device fault word.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+
+#include "attn_decode.cuh"
+#include "kv_ops.cuh"
+#include "pkv_internal.h"
+
+namespace {
+
+using pkv::fail;
+
+constexpr int kWarps = 4;    // consumer warps per decode CTA
+constexpr int kStages = 2;   // shared-memory stages per warp (one K+V block each)
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultPartitionTokens = 512;
+
+int elem_size(int32_t dtype) {
+    return dtype == PKV_F32 ? 4 : (dtype == PKV_F16 || dtype == PKV_BF16) ? 2 : 0;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Checks shared by every entry point that touches the pools.
+pkv_status check_pool_desc(const pkv_attn_desc *d, const char *fn) {
+    if (!d) return fail(PKV_ERR_INVALID, "%s: desc is NULL", fn);
+    if (!elem_size(d->dtype)) return fail(PKV_ERR_INVALID, "%s: unknown dtype %d", fn, d->dtype);
+    if (d->block_size != pkv::kBlock)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: block_size %d (only 16 is built)", fn,
+                    d->block_size);
+    if (d->head_dim != 64 && d->head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d (64 or 128)", fn, d->head_dim);
+    if (d->num_kv_heads < 1) return fail(PKV_ERR_INVALID, "%s: num_kv_heads < 1", fn);
+    if (d->num_blocks < 1) return fail(PKV_ERR_INVALID, "%s: num_blocks < 1", fn);
+    if ((int64_t)d->num_blocks * pkv::kBlock > INT64_MAX / 2)
+        return fail(PKV_ERR_INVALID, "%s: num_blocks too large", fn);
+    return PKV_OK;
+}
+
+struct Split {
+    int32_t part_blocks;
+    int32_t pmax;
+};
+
+pkv_status check_attn_desc(const pkv_attn_desc *d, const char *fn, Split *sp) {
+    pkv_status st = check_pool_desc(d, fn);
+    if (st) return st;
+    if (d->num_seqs < 0) return fail(PKV_ERR_INVALID, "%s: num_seqs < 0", fn);
+    if (d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads)
+        return fail(PKV_ERR_INVALID, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
+                    d->num_q_heads, d->num_kv_heads);
+    const int g = d->num_q_heads / d->num_kv_heads;
+    if (g != 1 && g != 2 && g != 4 && g != 8)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: query heads per kv head %d (1, 2, 4 or 8)", fn, g);
+    if (d->dtype == PKV_F32 && d->head_dim == 128 && g == 8)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: fp32 with head_dim 128 and group 8", fn);
+    if (d->max_blocks_per_seq < 1 || d->max_blocks_per_seq > INT_MAX / pkv::kBlock)
+        return fail(PKV_ERR_INVALID, "%s: max_blocks_per_seq %d", fn, d->max_blocks_per_seq);
+    if (d->partition_tokens < 0 || d->partition_tokens % pkv::kBlock)
+        return fail(PKV_ERR_INVALID, "%s: partition_tokens %d not a multiple of 16", fn,
+                    d->partition_tokens);
+    const int32_t pt = d->partition_tokens ? d->partition_tokens : kDefaultPartitionTokens;
+    sp->part_blocks = pt / pkv::kBlock;
+    sp->pmax = (d->max_blocks_per_seq + sp->part_blocks - 1) / sp->part_blocks;
+    const int64_t grid = (int64_t)d->num_seqs * d->num_kv_heads * sp->pmax;
+    if (grid > INT_MAX) return fail(PKV_ERR_INVALID, "%s: batch too large for one launch", fn);
+    return PKV_OK;
+}
+
+size_t workspace_bytes(const pkv_attn_desc *d, const Split &sp) {
+    if (sp.pmax <= 1) return 0;
+    const size_t rows = (size_t)d->num_seqs * d->num_q_heads * sp.pmax;
+    return round_up(rows * d->head_dim * sizeof(float), 256) + rows * 2 * sizeof(float);
+}
+
+pkv_status cuda_check(cudaError_t e, const char *fn, const char *what) {
+    if (e == cudaSuccess) return PKV_OK;
+    return fail(PKV_ERR_CUDA, "%s: %s: %s", fn, what, cudaGetErrorString(e));
+}
+
+// Opt each decode instantiation into its dynamic shared memory once per device.
+template <typename Kernel>
+pkv_status ensure_smem(Kernel kern, int bytes, std::atomic<bool> *done, const char *fn) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_check(e, fn, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_CUDA, "%s: device %d", fn, dev);
+    if (done[dev].load(std::memory_order_acquire)) return PKV_OK;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_check(e, fn, "cudaFuncSetAttribute");
+    done[dev].store(true, std::memory_order_release);
+    return PKV_OK;
+}
+
+template <typename T, int D, int G>
+pkv_status launch_decode(const pkv::DecodeParams &prm, cudaStream_t stream) {
+    using Cfg = pkv::DecodeCfg<T, D, G, kWarps, kStages>;
+    auto kern = pkv::paged_attn_decode_kernel<T, D, G, kWarps, kStages>;
+    static std::atomic<bool> done[kMaxDevices];
+    pkv_status st = ensure_smem(kern, Cfg::SMEM, done, "paged_attn_decode");
+    if (st) return st;
+    const unsigned grid = (unsigned)((int64_t)prm.S * prm.Hkv * prm.pmax);
+    kern<<<grid, kWarps * 32, Cfg::SMEM, stream>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "decode launch");
+    if (prm.pmax > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(((int64_t)prm.S * prm.Hq + 3) / 4));
+        cfg.blockDim = dim3(128);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, pkv::lse_reduce_kernel<T, D>, prm);
+        if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "reduce launch");
+    }
+    return PKV_OK;
+}
+
+template <typename T, int D>
+pkv_status dispatch_group(int g, const pkv::DecodeParams &prm, cudaStream_t stream) {
+    switch (g) {
+    case 1: return launch_decode<T, D, 1>(prm, stream);
+    case 2: return launch_decode<T, D, 2>(prm, stream);
+    case 4: return launch_decode<T, D, 4>(prm, stream);
+    case 8:
+        if constexpr (sizeof(T) == 4 && D == 128)
+            return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode: fp32, D 128, group 8");
+        else
+            return launch_decode<T, D, 8>(prm, stream);
+    default: return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode: group %d", g);
+    }
+}
+
+template <typename T>
+pkv_status dispatch_dim(int D, int g, const pkv::DecodeParams &prm, cudaStream_t stream) {
+    if (D == 64) return dispatch_group<T, 64>(g, prm, stream);
+    return dispatch_group<T, 128>(g, prm, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pkv_attn_workspace_bytes(const pkv_attn_desc *desc) {
+    pkv::clear_error();
+    Split sp;
+    if (check_attn_desc(desc, "pkv_attn_workspace_bytes", &sp)) return 0;
+    return workspace_bytes(desc, sp);
+}
+
+pkv_status paged_attn_decode(const pkv_attn_desc *desc, const void *q, const void *k_pool,
+                             const void *v_pool, const int32_t *block_tables,
+                             const int32_t *context_lens, float scale, void *out,
+                             void *workspace, size_t workspace_bytes_given, void *stream) {
+    const char *fn = "paged_attn_decode";
+    Split sp;
+    pkv_status st = check_attn_desc(desc, fn, &sp);
+    if (st) return st;
+    if (desc->num_seqs == 0) return PKV_OK;
+    if (!q || !k_pool || !v_pool || !block_tables || !context_lens || !out)
+        return fail(PKV_ERR_INVALID, "%s: NULL tensor pointer", fn);
+    if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16))
+        return fail(PKV_ERR_INVALID, "%s: q, pools and out must be 16-byte aligned", fn);
+    if (!aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return fail(PKV_ERR_INVALID, "%s: block_tables / context_lens misaligned", fn);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID, "%s: scale is not finite", fn);
+    const size_t need = workspace_bytes(desc, sp);
+    if (need) {
+        if (!workspace || workspace_bytes_given < need)
+            return fail(PKV_ERR_INVALID, "%s: workspace needs %zu bytes, got %zu", fn, need,
+                        workspace ? workspace_bytes_given : (size_t)0);
+        if (!aligned(workspace, 256))
+            return fail(PKV_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+    }
+    pkv::DecodeParams prm;
+    prm.q = q;
+    prm.k_pool = k_pool;
+    prm.v_pool = v_pool;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.out = out;
+    const size_t rows = (size_t)desc->num_seqs * desc->num_q_heads * sp.pmax;
+    prm.ws_o = need ? static_cast<float *>(workspace) : nullptr;
+    prm.ws_ml = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 round_up(rows * desc->head_dim * 4, 256))
+                     : nullptr;
+    prm.S = desc->num_seqs;
+    prm.Hq = desc->num_q_heads;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.maxB = desc->max_blocks_per_seq;
+    prm.part_blocks = sp.part_blocks;
+    prm.pmax = sp.pmax;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    const int g = desc->num_q_heads / desc->num_kv_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (desc->dtype) {
+    case PKV_F32: return dispatch_dim<float>(desc->head_dim, g, prm, s);
+    case PKV_F16: return dispatch_dim<__half>(desc->head_dim, g, prm, s);
+    default: return dispatch_dim<__nv_bfloat16>(desc->head_dim, g, prm, s);
+    }
+}
+
+pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
+                    const int64_t *slot_mapping, int32_t num_tokens, void *k_pool,
+                    void *v_pool, void *stream) {
+    const char *fn = "kv_write";
+    pkv_status st = check_pool_desc(desc, fn);
+    if (st) return st;
+    if (num_tokens < 0) return fail(PKV_ERR_INVALID, "%s: num_tokens < 0", fn);
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
+        return fail(PKV_ERR_INVALID, "%s: NULL tensor pointer", fn);
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pool, 16) ||
+        !aligned(v_pool, 16) || !aligned(slot_mapping, 8))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    pkv::KvWriteParams prm;
+    prm.k_new = static_cast<const uint4 *>(k_new);
+    prm.v_new = static_cast<const uint4 *>(v_new);
+    prm.slot_mapping = slot_mapping;
+    prm.k_pool = static_cast<uint4 *>(k_pool);
+    prm.v_pool = static_cast<uint4 *>(v_pool);
+    prm.T = num_tokens;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.vpr = desc->head_dim * elem_size(desc->dtype) / 16;
+    const int64_t total = 2LL * num_tokens * prm.Hkv * prm.vpr;
+    const int64_t blocks = (total + 255) / 256;
+    if (blocks > INT_MAX) return fail(PKV_ERR_INVALID, "%s: too many tokens", fn);
+    pkv::kv_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+    return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pairs,
+                          int32_t num_pairs, void *k_pool, void *v_pool, void *stream) {
+    const char *fn = "kv_copy_blocks";
+    pkv_status st = check_pool_desc(desc, fn);
+    if (st) return st;
+    if (num_pairs < 0) return fail(PKV_ERR_INVALID, "%s: num_pairs < 0", fn);
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_dst_pairs || !k_pool || !v_pool)
+        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
+    if (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(src_dst_pairs, 4))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    if (num_pairs > INT_MAX / 2) return fail(PKV_ERR_INVALID, "%s: too many pairs", fn);
+    pkv::KvCopyParams prm;
+    prm.pairs = src_dst_pairs;
+    prm.k_pool = static_cast<uint4 *>(k_pool);
+    prm.v_pool = static_cast<uint4 *>(v_pool);
+    prm.P = num_pairs;
+    prm.NB = desc->num_blocks;
+    prm.vpb = (int64_t)desc->num_kv_heads * pkv::kBlock * desc->head_dim *
+              elem_size(desc->dtype) / 16;
+    const int64_t slices = (prm.vpb + pkv::kCopyUnroll * 256 - 1) / (pkv::kCopyUnroll * 256);
+    if (slices > 65535) return fail(PKV_ERR_UNSUPPORTED, "%s: block too large", fn);
+    dim3 grid((unsigned)(2 * num_pairs), (unsigned)slices);
+    pkv::kv_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+    return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream) {
+    const char *fn = "pkv_device_faults";
+    if (!faults) return fail(PKV_ERR_INVALID, "%s: faults is NULL", fn);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int *addr = nullptr;
+    pkv_status st = cuda_check(cudaGetSymbolAddress((void **)&addr, pkv::g_faults), fn,
+                               "cudaGetSymbolAddress");
+    if (st) return st;
+    unsigned int h = 0;
+    st = cuda_check(cudaMemcpyAsync(&h, addr, sizeof(h), cudaMemcpyDeviceToHost, s), fn,
+                    "read");
+    if (st) return st;
+    if (clear) {
+        st = cuda_check(cudaMemsetAsync(addr, 0, sizeof(unsigned int), s), fn, "clear");
+        if (st) return st;
+    }
+    st = cuda_check(cudaStreamSynchronize(s), fn, "synchronize");
+    if (st) return st;
+    *faults = h;
+    return PKV_OK;
+}
+
+}  // extern "C"

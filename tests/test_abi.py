@@ -1,0 +1,118 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol include/pkv.h declares,
+and rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from paged_kv_cache_392_b200 import binding as B
+from paged_kv_cache_392_b200 import build as pbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
+    return sorted({n for n in names if n.startswith("pkv_") or n in (
+        "paged_attn_decode", "kv_write", "kv_copy_blocks")})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pbuild.build()
+    return B.lib()
+
+
+def test_header_declares_the_binding_exports():
+    assert header_functions() == sorted(B.EXPORTS)
+
+
+def test_library_exports_every_header_symbol(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", B.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_version_and_error_strings(lib):
+    assert "sm_100a" in B.version()
+    assert isinstance(B.last_error(), str)
+
+
+def _desc(**kw):
+    d = dict(num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=128, num_blocks=64,
+             max_blocks_per_seq=8, dtype=1, partition_tokens=0, block_size=16)
+    d.update(kw)
+    return B.AttnDesc(d["num_seqs"], d["num_q_heads"], d["num_kv_heads"], d["head_dim"],
+                      d["block_size"], d["num_blocks"], d["max_blocks_per_seq"],
+                      d["dtype"], d["partition_tokens"])
+
+
+def test_workspace_bytes(lib):
+    # 8 blocks * 16 = 128 tokens <= 512: one partition, no scratch
+    assert B.attn_workspace_bytes(_desc()) == 0
+    d = _desc(max_blocks_per_seq=100, partition_tokens=512)      # 1600 tokens: 4 parts
+    rows = 4 * 8 * 4
+    o = (rows * 128 * 4 + 255) // 256 * 256
+    assert B.attn_workspace_bytes(d) == o + rows * 2 * 4
+    with pytest.raises(B.PkvError):
+        B.attn_workspace_bytes(_desc(head_dim=80))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=96), 3), (dict(block_size=32), 3), (dict(num_q_heads=6), 3),
+    (dict(num_q_heads=7), 1), (dict(dtype=9), 1), (dict(num_blocks=0), 1),
+    (dict(partition_tokens=100), 1), (dict(max_blocks_per_seq=0), 1),
+    (dict(num_seqs=-1), 1), (dict(dtype=0, head_dim=128, num_q_heads=16), 3),
+])
+def test_decode_rejects_bad_descriptors_before_launch(lib, kw, code):
+    d = _desc(**kw)
+    fake = ctypes.c_void_p(1 << 20)
+    rc = lib.paged_attn_decode(ctypes.byref(d), fake, fake, fake, fake, fake, 0.1, fake,
+                               None, 0, None)
+    assert rc == code, B.last_error()
+    assert B.last_error()
+
+
+def test_decode_rejects_bad_pointers_and_workspace(lib):
+    d = _desc()
+    a = ctypes.c_void_p(1 << 20)
+    rc = lib.paged_attn_decode(ctypes.byref(d), None, a, a, a, a, 0.1, a, None, 0, None)
+    assert rc == 1 and "NULL" in B.last_error()
+    rc = lib.paged_attn_decode(ctypes.byref(d), ctypes.c_void_p((1 << 20) + 8), a, a, a, a,
+                               0.1, a, None, 0, None)
+    assert rc == 1 and "aligned" in B.last_error()
+    rc = lib.paged_attn_decode(ctypes.byref(d), a, a, a, a, a, float("nan"), a, None, 0, None)
+    assert rc == 1
+    d2 = _desc(max_blocks_per_seq=100, partition_tokens=512)
+    rc = lib.paged_attn_decode(ctypes.byref(d2), a, a, a, a, a, 0.1, a, None, 0, None)
+    assert rc == 1 and "workspace" in B.last_error()
+    rc = lib.paged_attn_decode(ctypes.byref(d2), a, a, a, a, a, 0.1, a,
+                               ctypes.c_void_p((1 << 20) + 16), 1 << 24, None)
+    assert rc == 1 and "256" in B.last_error()
+
+
+def test_empty_batches_launch_nothing(lib):
+    d = _desc(num_seqs=0)
+    assert lib.paged_attn_decode(ctypes.byref(d), None, None, None, None, None, 0.1, None,
+                                 None, 0, None) == 0
+    assert lib.kv_write(ctypes.byref(d), None, None, None, 0, None, None, None) == 0
+    assert lib.kv_copy_blocks(ctypes.byref(d), None, 0, None, None, None) == 0
+
+
+def test_kv_ops_reject_bad_arguments(lib):
+    d = _desc()
+    a = ctypes.c_void_p(1 << 20)
+    assert lib.kv_write(ctypes.byref(d), a, a, a, -1, a, a, None) == 1
+    assert lib.kv_write(ctypes.byref(d), a, None, a, 3, a, a, None) == 1
+    assert lib.kv_write(ctypes.byref(d), a, a, ctypes.c_void_p((1 << 20) + 4), 3, a, a,
+                        None) == 1
+    assert lib.kv_copy_blocks(ctypes.byref(d), None, 2, a, a, None) == 1
+    assert lib.kv_copy_blocks(ctypes.byref(_desc(head_dim=80)), a, 2, a, a, None) == 3
+    assert lib.pkv_device_faults(None, 0, None) == 1
