@@ -33,20 +33,22 @@ def up_to_date():
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force=False, verbose_ptxas=False):
-    """Compile libpkv.so unless it is newer than every source; return its path."""
-    if not force and up_to_date():
+def build(force=False, verbose_ptxas=False, out=None, defines=()):
+    """Compile libpkv.so unless it is newer than every source; return its path.
+    ``out``/``defines`` build a variant elsewhere (e.g. -DPKV_DECODE_WARPS=8)."""
+    target = out or LIB
+    if not force and out is None and up_to_date():
         return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = target + ".tmp.%d" % os.getpid()
     cmd = [NVCC] + ARCH + ["-lineinfo", "-O3", "-std=c++17", "-shared",
                            "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
                            "-I", os.path.join(ROOT, "include")]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
-    cmd += sources() + ["-o", tmp]
+    cmd += list(defines) + sources() + ["-o", tmp]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

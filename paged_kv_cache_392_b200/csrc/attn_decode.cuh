@@ -112,6 +112,28 @@ __device__ __forceinline__ void store_row(T *dst, const float (&x)[E]) {
     *reinterpret_cast<uint4 *>(dst) = u.v;
 }
 
+// Load G consecutive floats from shared memory (vectorised; p is 4*G-byte aligned).
+template <int G>
+__device__ __forceinline__ void load_g(const float *p, float (&x)[G]) {
+    if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < G; i += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(p + i);
+            x[i] = v.x;
+            x[i + 1] = v.y;
+            x[i + 2] = v.z;
+            x[i + 3] = v.w;
+        }
+    } else if constexpr (G == 2) {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        x[0] = v.x;
+        x[1] = v.y;
+    } else {
+#pragma unroll
+        for (int i = 0; i < G; ++i) x[i] = p[i];
+    }
+}
+
 template <typename T, int D, int G, int W, int NSW>
 struct DecodeCfg {
     static constexpr int ES = sizeof(T);
@@ -265,9 +287,9 @@ paged_attn_decode_kernel(const DecodeParams p) {
             Elem<T>::load(kv, kf);
 #pragma unroll
             for (int hh = 0; hh < G; ++hh) {
-                float a = 0.f;
+                float a = q[hh][0] * kf[0];
 #pragma unroll
-                for (int e = 0; e < E; ++e) a = fmaf(q[hh][e], kf[e], a);
+                for (int e = 1; e < E; ++e) a = fmaf(q[hh][e], kf[e], a);
                 v[ii * G + hh] = a;
             }
         }
@@ -323,11 +345,13 @@ paged_attn_decode_kernel(const DecodeParams p) {
         __syncwarp();
 
         // ---- P.V ----------------------------------------------------------------------
+        {
+            float alv[G];
+            load_g<G>(al, alv);
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-            const float a = al[hh];
+            for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-            for (int e = 0; e < E; ++e) o[hh][e] *= a;
+                for (int e = 0; e < E; ++e) o[hh][e] *= alv[hh];
         }
 #pragma unroll
         for (int ii = 0; ii < NPASS; ++ii) {
@@ -336,12 +360,12 @@ paged_attn_decode_kernel(const DecodeParams p) {
                 const uint4 vv = *reinterpret_cast<const uint4 *>(Vs + (t * CPR + c) * 16);
                 float vf[E];
                 Elem<T>::load(vv, vf);
+                float pr[G];
+                load_g<G>(sc + t * G, pr);
 #pragma unroll
-                for (int hh = 0; hh < G; ++hh) {
-                    const float pr = sc[t * G + hh];
+                for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-                    for (int e = 0; e < E; ++e) o[hh][e] = fmaf(pr, vf[e], o[hh][e]);
-                }
+                    for (int e = 0; e < E; ++e) o[hh][e] = fmaf(pr[hh], vf[e], o[hh][e]);
             }
         }
         __syncwarp();

@@ -14,8 +14,14 @@ namespace {
 
 using pkv::fail;
 
-constexpr int kWarps = 4;    // consumer warps per decode CTA
-constexpr int kStages = 2;   // shared-memory stages per warp (one K+V block each)
+#ifndef PKV_DECODE_WARPS
+#define PKV_DECODE_WARPS 4
+#endif
+#ifndef PKV_DECODE_STAGES
+#define PKV_DECODE_STAGES 2
+#endif
+constexpr int kWarps = PKV_DECODE_WARPS;    // consumer warps per decode CTA
+constexpr int kStages = PKV_DECODE_STAGES;  // shared-memory stages per warp (K+V block each)
 constexpr int kMaxDevices = 64;
 constexpr int kDefaultPartitionTokens = 512;
 

@@ -106,7 +106,9 @@ def test_split_and_unsplit_agree_closely():
     wl = small_wl([3000, 1800, 4096], 4, 4, 128, "f32", seed=5)
     vals = W.make_values(wl, "cpu")
     a, ref = run_step(wl, vals, partition_tokens=64)
-    b, _ = run_step(wl, vals, partition_tokens=4096, write=False)
+    # unsplit: 256 blocks per work unit, 64 per warp (more than one table chunk of 32)
+    b, ref_b = run_step(wl, vals, partition_tokens=4096)
+    assert np.array_equal(ref, ref_b)
     assert np.max(np.abs(a - ref)) <= 1e-5 and np.max(np.abs(b - ref)) <= 1e-5
 
 
