@@ -134,6 +134,32 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
                           int32_t num_pairs, void *k_pool, void *v_pool, void *stream);
 
 /*
+ * Allocation-free variant of paged_attn_decode.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- for example a serving
+ * engine that hands (nearly) all free HBM to its KV pool at start-up and owns every later
+ * allocation, a plugin or custom-op interface whose host framework forbids allocating inside
+ * the op, or a latency-critical loop where cudaMalloc/cudaFree would synchronise the device.
+ * It takes the same arguments as paged_attn_decode minus the workspace, and keeps the
+ * split-context partial results in a scratch array that is part of the library itself:
+ * PKV_STATIC_WORKSPACE_BYTES of device memory, held on every GPU that loads the library
+ * until the process exits.  It calls no allocating routine.
+ *   - The first call on a device looks up that device's copy of the array (once per
+ *     device, with that device current); make that first call before any stream capture.
+ *   - A batch whose split scratch (pkv_attn_workspace_bytes) exceeds
+ *     PKV_STATIC_WORKSPACE_BYTES is rejected with PKV_ERR_INVALID; nothing is launched.
+ *   - Every call on a device shares the one array and it keeps the last call's contents
+ *     (nothing in it needs to start at zero: each partial is written before it is read).
+ *     Calls whose work overlaps on the GPU (other streams, other host threads) race on it:
+ *     order them on one stream, or use paged_attn_decode with a workspace per stream.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (32u << 20)
+pkv_status paged_attn_decode_no_alloc(const pkv_attn_desc *desc, const void *q,
+                                      const void *k_pool, const void *v_pool,
+                                      const int32_t *block_tables,
+                                      const int32_t *context_lens, float scale, void *out,
+                                      void *stream);
+
+/*
  * Read the device fault word of the current device into *faults (host) after the work
  * queued on stream so far has finished; clear != 0 resets it to 0.  Synchronises stream.
  */

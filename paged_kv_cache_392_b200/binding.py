@@ -24,7 +24,7 @@ BLOCK_SIZE = 16
 # Every symbol include/pkv.h declares.
 EXPORTS = [
     "pkv_last_error", "pkv_version", "pkv_attn_workspace_bytes", "paged_attn_decode",
-    "kv_write", "kv_copy_blocks", "pkv_device_faults", "pkv_bm_create", "pkv_bm_destroy",
+    "kv_write", "kv_copy_blocks", "pkv_device_faults", "paged_attn_decode_no_alloc", "pkv_bm_create", "pkv_bm_destroy",
     "pkv_bm_add_seq", "pkv_bm_append_slot", "pkv_bm_append_slots", "pkv_bm_fork",
     "pkv_bm_free_seq", "pkv_bm_block_table", "pkv_bm_block_tables", "pkv_bm_seq_len",
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
@@ -67,6 +67,7 @@ def lib():
         "pkv_version": ([], ctypes.c_char_p),
         "pkv_attn_workspace_bytes": ([dp], sz),
         "paged_attn_decode": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz, vp], i32),
+        "paged_attn_decode_no_alloc": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
         "kv_write": ([dp, vp, vp, vp, i32, vp, vp, vp], i32),
         "kv_copy_blocks": ([dp, vp, i32, vp, vp, vp], i32),
         "pkv_device_faults": ([P(ctypes.c_uint32), ctypes.c_int, vp], i32),
@@ -191,6 +192,28 @@ def paged_attn_decode(q, k_pool, v_pool, block_tables, context_lens, scale, out=
                                    _ptr(block_tables), _ptr(context_lens), float(scale),
                                    _ptr(out), _ptr(workspace), nbytes,
                                    _stream(stream, q.device)))
+    return out
+
+
+STATIC_WORKSPACE_BYTES = 32 << 20   # PKV_STATIC_WORKSPACE_BYTES in include/pkv.h
+
+
+def paged_attn_decode_no_alloc(q, k_pool, v_pool, block_tables, context_lens, scale,
+                               out, partition_tokens=0, stream=None):
+    """paged_attn_decode for callers that cannot allocate device memory: the split scratch
+    lives in the library's own static device array (STATIC_WORKSPACE_BYTES per GPU) and
+    ``out`` must be given.  Calls that overlap on the GPU share that array and race."""
+    _dev(q, "q", k_pool.dtype)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    _dev(out, "out", q.dtype)
+    if q.dim() != 3 or out.shape != q.shape or block_tables.dim() != 2 or \
+            block_tables.shape[0] != q.shape[0] or context_lens.shape != (q.shape[0],):
+        raise ValueError("q/out [S,Hq,D], block_tables [S,maxB], context_lens [S] expected")
+    desc = decode_desc(q, k_pool, v_pool, block_tables, partition_tokens)
+    _check(lib().paged_attn_decode_no_alloc(
+        ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
+        _ptr(context_lens), float(scale), _ptr(out), _stream(stream, q.device)))
     return out
 
 

@@ -5,6 +5,7 @@
 #include <atomic>
 #include <climits>
 #include <cmath>
+#include <mutex>
 
 #include "attn_decode.cuh"
 #include "kv_ops.cuh"
@@ -272,6 +273,67 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
     dim3 grid((unsigned)(2 * num_pairs), (unsigned)slices);
     pkv::kv_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
     return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+}  // extern "C"
+
+// ---- allocation-free decode ----------------------------------------------------------------
+// Split-context scratch that ships inside the library: one copy per device that loads it.
+// In host code the name below is only a host-side stand-in for the device array, never a
+// device address; the device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_static_workspace[PKV_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+std::mutex g_static_ws_mutex;
+void *g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of the current device's copy of g_static_workspace (looked up on first use).
+pkv_status static_workspace(void **ptr, const char *fn) {
+    int dev = 0;
+    pkv_status st = cuda_check(cudaGetDevice(&dev), fn, "cudaGetDevice");
+    if (st) return st;
+    if (dev < 0 || dev >= kMaxDevices) return fail(PKV_ERR_CUDA, "%s: device %d", fn, dev);
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_ptr[dev]) {
+        void *p = nullptr;
+        st = cuda_check(cudaGetSymbolAddress(&p, g_static_workspace), fn,
+                        "cudaGetSymbolAddress(static workspace)");
+        if (st) return st;
+        g_static_ws_ptr[dev] = p;
+    }
+    *ptr = g_static_ws_ptr[dev];
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status paged_attn_decode_no_alloc(const pkv_attn_desc *desc, const void *q,
+                                      const void *k_pool, const void *v_pool,
+                                      const int32_t *block_tables,
+                                      const int32_t *context_lens, float scale, void *out,
+                                      void *stream) {
+    const char *fn = "paged_attn_decode_no_alloc";
+    Split sp;
+    pkv_status st = check_attn_desc(desc, fn, &sp);
+    if (st) return st;
+    const size_t need = workspace_bytes(desc, sp);
+    if (need > PKV_STATIC_WORKSPACE_BYTES)
+        return fail(PKV_ERR_INVALID,
+                    "%s: this batch needs %zu bytes of split scratch; the library's static "
+                    "workspace holds %u (use paged_attn_decode with a workspace, fewer "
+                    "sequences, or larger partition_tokens)",
+                    fn, need, (unsigned)PKV_STATIC_WORKSPACE_BYTES);
+    if (desc->num_seqs == 0) return PKV_OK;
+    void *ws = nullptr;
+    if (need) {
+        st = static_workspace(&ws, fn);
+        if (st) return st;
+    }
+    return paged_attn_decode(desc, q, k_pool, v_pool, block_tables, context_lens, scale, out,
+                             ws, need ? (size_t)PKV_STATIC_WORKSPACE_BYTES : 0, stream);
 }
 
 pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream) {

@@ -18,8 +18,8 @@ def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
-    return sorted({n for n in names if n.startswith("pkv_") or n in (
-        "paged_attn_decode", "kv_write", "kv_copy_blocks")})
+    return sorted({n for n in names if n.startswith(("pkv_", "paged_attn_decode")) or n in (
+        "kv_write", "kv_copy_blocks")})
 
 
 @pytest.fixture(scope="module")
