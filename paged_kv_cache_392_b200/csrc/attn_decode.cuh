@@ -134,6 +134,53 @@ __device__ __forceinline__ void load_g(const float *p, float (&x)[G]) {
     }
 }
 
+// Merge the W warps' (max, sum, unnormalised output) states of one work unit from shared
+// memory (mo [W][G][D], mml [W][G][2], base-2 units) and write either the normalised output
+// (the unit covers the whole sequence) or the unit's partial state for the reduce kernel.
+// Called by all W*32 threads after a __syncthreads().
+template <typename T, int D, int G, int W>
+__device__ __forceinline__ void merge_and_store(const DecodeParams &p, const float *mo,
+                                                const float *mml, int s, int hk, int part,
+                                                int nparts) {
+    constexpr int E = 16 / sizeof(T);
+    constexpr int VPH = D / E;  // 16-byte output vectors per head
+    for (int idx = threadIdx.x; idx < G * VPH; idx += W * 32) {
+        const int hh = idx / VPH;
+        const int d0 = (idx % VPH) * E;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < W; ++w) M = fmaxf(M, mml[(w * G + hh) * 2]);
+        float den = 0.f, num[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) num[e] = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const float mw = mml[(w * G + hh) * 2];
+            const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            den += a * mml[(w * G + hh) * 2 + 1];
+#pragma unroll
+            for (int e = 0; e < E; ++e) num[e] += a * mo[(w * G + hh) * D + d0 + e];
+        }
+        const int h = hk * G + hh;
+        if (nparts == 1) {
+            const float inv = 1.f / den;
+#pragma unroll
+            for (int e = 0; e < E; ++e) num[e] *= inv;
+            store_row<T, E>(static_cast<T *>(p.out) + ((size_t)s * p.Hq + h) * D + d0, num);
+        } else {
+            const size_t row = ((size_t)s * p.Hq + h) * p.pmax + part;
+            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D + d0);
+#pragma unroll
+            for (int e = 0; e < E; e += 4)
+                dst[e / 4] = make_float4(num[e], num[e + 1], num[e + 2], num[e + 3]);
+            if (d0 == 0) {
+                p.ws_ml[row * 2] = M;
+                p.ws_ml[row * 2 + 1] = den;
+            }
+        }
+    }
+}
+
 template <typename T, int D, int G, int W, int NSW>
 struct DecodeCfg {
     static constexpr int ES = sizeof(T);
@@ -415,43 +462,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
     }
     __syncthreads();
 
-    // ---- merge the W warps; write output or this partition's partial state -------------
-    constexpr int VPH = D / E;  // 16-byte output vectors per head
-    for (int idx = threadIdx.x; idx < G * VPH; idx += W * 32) {
-        const int hh = idx / VPH;
-        const int d0 = (idx % VPH) * E;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < W; ++w) M = fmaxf(M, mml[(w * G + hh) * 2]);
-        float den = 0.f, num[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) num[e] = 0.f;
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-            const float mw = mml[(w * G + hh) * 2];
-            const float a = mw == -INFINITY ? 0.f : exp2f(mw - M);
-            den += a * mml[(w * G + hh) * 2 + 1];
-#pragma unroll
-            for (int e = 0; e < E; ++e) num[e] += a * mo[(w * G + hh) * D + d0 + e];
-        }
-        const int h = hk * G + hh;
-        if (nparts == 1) {
-            const float inv = 1.f / den;
-#pragma unroll
-            for (int e = 0; e < E; ++e) num[e] *= inv;
-            store_row<T, E>(static_cast<T *>(p.out) + ((size_t)s * p.Hq + h) * D + d0, num);
-        } else {
-            const size_t row = ((size_t)s * p.Hq + h) * p.pmax + part;
-            float4 *dst = reinterpret_cast<float4 *>(p.ws_o + row * D + d0);
-#pragma unroll
-            for (int e = 0; e < E; e += 4)
-                dst[e / 4] = make_float4(num[e], num[e + 1], num[e + 2], num[e + 3]);
-            if (d0 == 0) {
-                p.ws_ml[row * 2] = M;
-                p.ws_ml[row * 2 + 1] = den;
-            }
-        }
-    }
+    merge_and_store<T, D, G, W>(p, mo, mml, s, hk, part, nparts);
 }
 
 // ---- log-sum-exp merge of the partitions of split sequences ----------------------------

@@ -1,5 +1,7 @@
 // Host side of libpkv's CUDA path: argument validation, kernel selection and launches for
 // paged_attn_decode, kv_write and kv_copy_blocks, plus the device fault word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -8,6 +10,7 @@
 #include <mutex>
 
 #include "attn_decode.cuh"
+#include "attn_decode_tc.cuh"
 #include "kv_ops.cuh"
 #include "pkv_internal.h"
 
@@ -105,6 +108,88 @@ pkv_status ensure_smem(Kernel kern, int bytes, std::atomic<bool> *done, const ch
     return PKV_OK;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no libcuda
+// link dependency).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// 2-D view [rows = NB*H_kv*16][D] of a 16-bit pool, boxes of 16 rows x 64 columns (128 B)
+// with the 128-byte swizzle.
+pkv_status kv_tensor_map(CUtensorMap *m, const void *pool, int32_t dtype, int D, int64_t rows,
+                         const char *fn) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(PKV_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", fn);
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)pkv::kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     2, const_cast<void *>(pool), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PKV_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", fn, (int)r);
+    return PKV_OK;
+}
+
+pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t stream,
+                                  void (*kern)(const pkv::DecodeParams)) {
+    if (prm.pmax <= 1) return PKV_OK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(((int64_t)prm.S * prm.Hq + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    return cuda_check(e, "paged_attn_decode", "reduce launch");
+}
+
+#ifndef PKV_DECODE_TC_WARPS
+#define PKV_DECODE_TC_WARPS 2
+#endif
+#ifndef PKV_DECODE_TC_STAGES
+#define PKV_DECODE_TC_STAGES 2
+#endif
+constexpr int kTcWarps = PKV_DECODE_TC_WARPS;
+constexpr int kTcStages = PKV_DECODE_TC_STAGES;
+
+// Tensor-core decode for 16-bit K/V.
+template <typename T, int D, int G>
+pkv_status launch_decode_tc(const pkv::DecodeParams &prm, int32_t dtype, cudaStream_t stream) {
+    using Cfg = pkv::DecodeTcCfg<T, D, G, kTcWarps, kTcStages>;
+    auto kern = pkv::paged_attn_decode_tc_kernel<T, D, G, kTcWarps, kTcStages>;
+    static std::atomic<bool> done[kMaxDevices];
+    pkv_status st = ensure_smem(kern, Cfg::SMEM, done, "paged_attn_decode");
+    if (st) return st;
+    const int64_t rows = (int64_t)prm.NB * prm.Hkv * pkv::kBlock;
+    CUtensorMap tmk, tmv;
+    st = kv_tensor_map(&tmk, prm.k_pool, dtype, D, rows, "paged_attn_decode");
+    if (st) return st;
+    st = kv_tensor_map(&tmv, prm.v_pool, dtype, D, rows, "paged_attn_decode");
+    if (st) return st;
+    const unsigned grid = (unsigned)((int64_t)prm.S * prm.Hkv * prm.pmax);
+    kern<<<grid, kTcWarps * 32, Cfg::SMEM, stream>>>(tmk, tmv, prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "decode launch");
+    return launch_reduce_if_split(prm, stream, pkv::lse_reduce_kernel<T, D>);
+}
+
 template <typename T, int D, int G>
 pkv_status launch_decode(const pkv::DecodeParams &prm, cudaStream_t stream) {
     using Cfg = pkv::DecodeCfg<T, D, G, kWarps, kStages>;
@@ -131,6 +216,30 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, cudaStream_t stream) {
         if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "reduce launch");
     }
     return PKV_OK;
+}
+
+// Whether the tensor-core kernel serves this call: 16-bit K/V whose 2-D TMA view fits int32
+// row coordinates.  PKV_DECODE_FORCE_SIMT builds keep every call on the CUDA-core kernel.
+bool use_tc(const pkv_attn_desc *d) {
+#ifdef PKV_DECODE_FORCE_SIMT
+    (void)d;
+    return false;
+#else
+    return d->dtype != PKV_F32 &&
+           (int64_t)d->num_blocks * d->num_kv_heads * pkv::kBlock < ((int64_t)1 << 31);
+#endif
+}
+
+template <typename T, int D>
+pkv_status dispatch_group_tc(int g, const pkv::DecodeParams &prm, int32_t dtype,
+                             cudaStream_t stream) {
+    switch (g) {
+    case 1: return launch_decode_tc<T, D, 1>(prm, dtype, stream);
+    case 2: return launch_decode_tc<T, D, 2>(prm, dtype, stream);
+    case 4: return launch_decode_tc<T, D, 4>(prm, dtype, stream);
+    case 8: return launch_decode_tc<T, D, 8>(prm, dtype, stream);
+    default: return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode: group %d", g);
+    }
 }
 
 template <typename T, int D>
@@ -211,6 +320,14 @@ pkv_status paged_attn_decode(const pkv_attn_desc *desc, const void *q, const voi
     prm.scale_log2 = scale * 1.4426950408889634f;
     const int g = desc->num_q_heads / desc->num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_tc(desc)) {
+        if (desc->dtype == PKV_F16)
+            return desc->head_dim == 64 ? dispatch_group_tc<__half, 64>(g, prm, PKV_F16, s)
+                                        : dispatch_group_tc<__half, 128>(g, prm, PKV_F16, s);
+        return desc->head_dim == 64
+                   ? dispatch_group_tc<__nv_bfloat16, 64>(g, prm, PKV_BF16, s)
+                   : dispatch_group_tc<__nv_bfloat16, 128>(g, prm, PKV_BF16, s);
+    }
     switch (desc->dtype) {
     case PKV_F32: return dispatch_dim<float>(desc->head_dim, g, prm, s);
     case PKV_F16: return dispatch_dim<__half>(desc->head_dim, g, prm, s);
