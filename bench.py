@@ -33,6 +33,8 @@ METRIC = "paged decode attention KV GB/s & seqs/s, % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
 
 WORKLOAD_TEXT = {
+    "tiny": "tiny decode step: 4 seqs, context {5,17,33,48}, 2 heads MHA, head_dim 64, fp32, "
+            "block 16, 16-block pool, kv_write of one token per sequence",
     "opt13b": "OPT-13B-shaped decode: 64 seqs, 40 heads MHA, head_dim 128, fp16 KV, block 16, "
               "context lognormal(median 512, sigma 1) clipped 16..2048, shuffled placement, "
               "pool 1.1x need, kv_write of one token per sequence",
@@ -56,6 +58,11 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--read-probe", action="store_true",
+                    help="also measure a read-only streaming ceiling (torch.sum, 2 GiB)")
+    ap.add_argument("--contiguous", action="store_true",
+                    help="place each sequence's blocks contiguously and in order (paged "
+                         "kernel over a contiguous layout) instead of shuffled")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
@@ -128,6 +135,22 @@ class _ModelAdapter:
 
     def close(self):
         pass
+
+
+def contiguous_placement(wl):
+    """Re-place every sequence's blocks back to back in pool order (block j of sequence s at
+    pool block off_s + j): the layout a contiguous cache would have, read through the same
+    block tables by the same kernel."""
+    nblk = (wl.context_lens.astype(np.int64) + 15) // 16
+    bt = np.full_like(wl.block_tables, -1)
+    off = 0
+    for s_, n in enumerate(nblk):
+        bt[s_, :n] = np.arange(off, off + n, dtype=np.int32)
+        off += n
+    wl.block_tables = bt
+    pos = wl.context_lens.astype(np.int64) - 1
+    wl.slot_mapping = bt[np.arange(wl.num_seqs), pos // 16].astype(np.int64) * 16 + pos % 16
+    wl.extra["placement"] = "contiguous"
 
 
 def algorithmic_bytes(wl, pairs, split_rows=0, pmax_used=None):
@@ -279,6 +302,23 @@ def barrier(dist, device):
             dist.barrier()
 
 
+def read_probe_gbs(torch, device, gib=2, reps=5):
+    """Best-of-reps read bandwidth of a plain streaming reduction (torch.sum over a 2 GiB
+    bf16 buffer): a read-only ceiling to set beside the copy-based peak."""
+    x = torch.ones(gib << 29, dtype=torch.bfloat16, device=device)
+    best = 0.0
+    for _ in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum(dtype=torch.float32)
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, x.numel() * 2 / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del x
+    torch.cuda.empty_cache()
+    return round(best, 1)
+
+
 # ---- the CUDA path --------------------------------------------------------------------------
 def gpu_uuid(torch, device):
     try:
@@ -301,6 +341,10 @@ def run_pkv(args):
     dist = init_dist(world)
 
     wl, pairs = build_workload(args.workload)
+    if args.contiguous:
+        if args.workload == "fork":
+            raise SystemExit("--contiguous does not apply to the fork workload")
+        contiguous_placement(wl)
     pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens
     vals = W.make_values(wl, device)
     q, kp, vp, kn, vn = (vals[k] for k in ("q", "k_pool", "v_pool", "k_new", "v_new"))
@@ -332,26 +376,48 @@ def run_pkv(args):
     if faults:
         raise RuntimeError("device faults during warm-up: %s" % faults)
 
+    # Runs of N consecutive steps are captured as one CUDA graph on a side stream, with an
+    # event-record node on each side of every decode call; the timed loop replays the
+    # graph, so neither host launch overhead nor gaps between launches leak into device
+    # time.  The decode-call durations come from those events (the last replay's N calls).
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
+    N = max(1, min(50, K))
+    gs = torch.cuda.Stream(device)
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(N)]
+
+    def capture(nsteps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for j in range(nsteps):
+                if npairs:
+                    B.kv_copy_blocks(pairs_d, kp, vp)
+                B.kv_write(kn, vn, slots, kp, vp)
+                ev[j][0].record(gs)
+                B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
+                                    partition_tokens=pt)
+                ev[j][1].record(gs)
+        return g
+
+    g_run = capture(N)
+    g_rem = capture(K % N) if K % N else None
+    torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(gpu_uuid(torch, device))
-    barrier(dist, device)
-    torch.cuda.synchronize()
-    sampler.start()
-    t0.record()
-    for i in range(K):
-        if npairs:
-            B.kv_copy_blocks(pairs_d, kp, vp)
-        B.kv_write(kn, vn, slots, kp, vp)
-        ev[i][0].record()
-        B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
-                            partition_tokens=pt)
-        ev[i][1].record()
-    t1.record()
-    torch.cuda.synchronize()
-    barrier(dist, device)
+    with torch.cuda.stream(gs):
+        for _ in range(max(1, -(-args.warmup // N))):
+            g_run.replay()
+        barrier(dist, device)
+        torch.cuda.synchronize()
+        sampler.start()
+        t0.record(gs)
+        if g_rem is not None:
+            g_rem.replay()
+        for _ in range(K // N):
+            g_run.replay()
+        t1.record(gs)
+        torch.cuda.synchronize()
+        barrier(dist, device)
     sampler.stop()
     ms_local = t0.elapsed_time(t1)
     ms = max_over_ranks(dist, ms_local, device)
@@ -360,42 +426,120 @@ def run_pkv(args):
     faults = B.device_faults(clear=True)
     if faults:
         raise RuntimeError("device faults during timing: %s" % faults)
+    del g_run, g_rem
 
     # ---- end to end through the public API with host buffers -------------------------
-    pin = {k: v.cpu().pin_memory() for k, v in (("q", q), ("kn", kn), ("vn", vn),
-                                                 ("slots", slots), ("bt", bt),
-                                                 ("lens", lens), ("pairs", pairs_d))}
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = out_h.numel() * out_h.element_size()
-    stream = torch.cuda.current_stream(device)
+    # Every step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs) from pinned
+    # host memory and reads its output back.  "serial": one step at a time, synchronised.
+    # "pipelined": two input buffer sets; the copies of step i+1 run on a copy stream while
+    # step i computes, and the host waits for each step's output one step behind.
+    host_in = {"q": q, "kn": kn, "vn": vn, "slots": slots, "bt": bt, "lens": lens,
+               "pairs": pairs_d}
+    pin = {k: v.cpu().pin_memory() for k, v in host_in.items()}
+    h2d = sum(t.numel() * t.element_size() for k, t in pin.items()
+              if k != "pairs" or npairs)
+    d2h = out.numel() * out.element_size()
+    torch.cuda.synchronize()
+    main = torch.cuda.Stream(device)          # graphs are captured on non-default streams
+    copy_stream = torch.cuda.Stream(device)
+    bufs = [host_in, {k: v.clone() for k, v in host_in.items()}]
+    outs = [out, torch.empty_like(out)]
+    outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    used = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        q.copy_(pin["q"], non_blocking=True)
-        kn.copy_(pin["kn"], non_blocking=True)
-        vn.copy_(pin["vn"], non_blocking=True)
-        slots.copy_(pin["slots"], non_blocking=True)
-        bt.copy_(pin["bt"], non_blocking=True)
-        lens.copy_(pin["lens"], non_blocking=True)
+    def run_kernels(b):
+        d = bufs[b]
         if npairs:
-            pairs_d.copy_(pin["pairs"], non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
-        stream.synchronize()
+            B.kv_copy_blocks(d["pairs"], kp, vp)
+        B.kv_write(d["kn"], d["vn"], d["slots"], kp, vp)
+        B.paged_attn_decode(d["q"], kp, vp, d["bt"], d["lens"], wl.scale, out=outs[b],
+                            workspace=ws, partition_tokens=pt)
 
+    def h2d_copy(b, stream):
+        with torch.cuda.stream(stream):
+            for k, t in bufs[b].items():
+                if k != "pairs" or npairs:
+                    t.copy_(pin[k], non_blocking=True)
+
+    def e2e_serial_step():
+        with torch.cuda.stream(main):
+            h2d_copy(0, main)
+            run_kernels(0)
+            outs_h[0].copy_(outs[0], non_blocking=True)
+        main.synchronize()
+
+    # Each half of a step (the input copies; the kernels plus the output copy) is captured
+    # once per buffer set as a CUDA graph, so a step costs the host two graph launches.
+    g_copy, g_comp = [], []
+    for b in range(2):
+        with torch.cuda.stream(main):
+            run_kernels(b)                 # warm the library paths outside capture
+        main.synchronize()
+        gc = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gc, stream=copy_stream):
+            for k, t in bufs[b].items():
+                if k != "pairs" or npairs:
+                    t.copy_(pin[k], non_blocking=True)
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gk, stream=main):
+            run_kernels(b)
+        g_copy.append(gc)
+        g_comp.append(gk)
+    torch.cuda.synchronize()
+    d2h_stream = torch.cuda.Stream(device)
+    k_done = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_pipelined(n):
+        with torch.cuda.stream(copy_stream):
+            g_copy[0].replay()
+        h2d_done[0].record(copy_stream)
+        for i in range(n):
+            b = i & 1
+            if i + 1 < n:          # stage the next step's inputs behind its buffer's last use
+                nb = (i + 1) & 1
+                copy_stream.wait_event(used[nb])
+                with torch.cuda.stream(copy_stream):
+                    g_copy[nb].replay()
+                h2d_done[nb].record(copy_stream)
+            main.wait_event(h2d_done[b])
+            with torch.cuda.stream(main):
+                g_comp[b].replay()
+            k_done[b].record(main)
+            d2h_stream.wait_event(k_done[b])      # output copy off the compute stream
+            with torch.cuda.stream(d2h_stream):
+                outs_h[b].copy_(outs[b], non_blocking=True)
+            used[b].record(d2h_stream)
+            if i >= 1:
+                used[(i - 1) & 1].synchronize()   # host has step i-1's output
+        d2h_stream.synchronize()
+        main.synchronize()
+
+    Ke = max(1, K)                # same number of steps as the device loop (same power state)
+    Ks = max(1, min(K, 1000))     # serial mode: at most 1000 synchronised steps
     for _ in range(max(3, args.warmup // 4)):
-        e2e_step()
-    Ke = max(1, min(K, 500))
+        e2e_serial_step()
+    e2e_pipelined(4)
     barrier(dist, device)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(Ke):
-        e2e_step()
-    e1.record()
+    e0.record(main)
+    for _ in range(Ks):
+        e2e_serial_step()
+    e1.record(main)
+    torch.cuda.synchronize()
+    e2e_serial_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ks, device)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    e0.record(main)
+    e2e_pipelined(Ke)
+    e1.record(main)                # e2e_pipelined returned after the last output landed
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ke, device)
     barrier(dist, device)
+    faults = B.device_faults(clear=True)
+    if faults:
+        raise RuntimeError("device faults during the end-to-end runs: %s" % faults)
 
     result = None
     if rank == 0:
@@ -404,6 +548,7 @@ def run_pkv(args):
         kv_gbs = world * nbytes["kv"] / (step_ms * 1e-3) / 1e9
         achieved = nbytes["decode"] / (decode_ms * 1e-3) / 1e9
         traffic = profile_traffic(args.workload)
+        probe = read_probe_gbs(torch, device) if args.read_probe else None
         result = {
             "metric": METRIC,
             "value": round(kv_gbs, 2),
@@ -431,6 +576,7 @@ def run_pkv(args):
                 "l2": "no flush: KV working set %.2f GB per step > 126 MB L2" %
                       (nbytes["kv"] / 1e9),
                 "parallelism": "replicas x%d" % world,
+                "placement": wl.extra.get("placement", "shuffled"),
             },
             "roofline": {
                 "bound": "hbm",
@@ -441,6 +587,8 @@ def run_pkv(args):
                 "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
+                "read_probe_gbs": probe,
+                "frac_of_read_probe": round(achieved / probe, 4) if probe else None,
                 "traffic": traffic,
                 "algorithmic_bytes": nbytes["decode"],
                 "avg_launch_ms": round(decode_ms, 5),
@@ -448,7 +596,13 @@ def run_pkv(args):
             "e2e": {"value": round(world * nbytes["kv"] / (e2e_ms * 1e-3) / 1e9, 2),
                     "unit": "GB/s", "ms_per_step": round(e2e_ms, 5),
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "steps": Ke},
+                    "steps": Ke, "mode": "pipelined: input copies of step i+1 and the output "
+                                          "copy of step i-1 overlap step i's kernels "
+                                          "(three streams, kernels and input copies "
+                                          "replayed as CUDA graphs)",
+                    "serial_value": round(world * nbytes["kv"] / (e2e_serial_ms * 1e-3) / 1e9,
+                                          2),
+                    "serial_ms_per_step": round(e2e_serial_ms, 5)},
             "gpu_launches": K * launches_per_step,
             "clocks": sampler.summary(),
         }

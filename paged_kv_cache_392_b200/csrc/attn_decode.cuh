@@ -467,14 +467,24 @@ paged_attn_decode_kernel(const DecodeParams p) {
 
 // ---- log-sum-exp merge of the partitions of split sequences ----------------------------
 // out[s,h,:] = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p  (base-2 units,
-// which is the natural-log formula with every logit scaled by log2(e)).  One warp per row;
-// rows whose sequence fits in one partition were already written by the decode kernel.
+// which is the natural-log formula with every logit scaled by log2(e)).  One CTA of four
+// warps per (sequence, query head) row: the warps take every fourth partition, each lane a
+// D/32-float slice of o_p (vector loads, unrolled so several partitions are in flight), and
+// the four partial sums meet in shared memory.  Rows whose sequence fits in one partition
+// were already written by the decode kernel.
+constexpr int kReduceWarps = 4;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams p) {
-    constexpr int DPL = D / 32;  // elements per lane
+__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const DecodeParams p) {
+    constexpr int NW = kReduceWarps;
+    constexpr int VL = D / 32;             // floats per lane
+    constexpr int E = 16 / sizeof(T);      // output elements per 16-byte store
+    __shared__ float s_m[NW];
+    __shared__ float s_den[NW];
+    __shared__ __align__(16) float s_acc[NW][D];
+
     pdl_wait_primary();
-    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x;
     if (row >= p.S * p.Hq) return;
     const int s = row / p.Hq;
     const int L = p.context_lens[s];
@@ -484,29 +494,57 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams p) {
     if (np <= 1) return;
     const float *ml = p.ws_ml + (size_t)row * p.pmax * 2;
     const float *ob = p.ws_o + (size_t)row * p.pmax * D;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, ml[2 * i]);
+    for (int i = threadIdx.x; i < np; i += NW * 32) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    float den = 0.f;
-    for (int i = lane; i < np; i += 32) den += exp2f(ml[2 * i] - M) * ml[2 * i + 1];
+    if (lane == 0) s_m[warp] = M;
+    __syncthreads();
 #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w]);
 
-    float acc[DPL];
+    float acc[VL], den = 0.f;
 #pragma unroll
-    for (int k = 0; k < DPL; ++k) acc[k] = 0.f;
-    for (int i = 0; i < np; ++i) {
+    for (int k = 0; k < VL; ++k) acc[k] = 0.f;
+#pragma unroll 4
+    for (int i = warp; i < np; i += NW) {
         const float w = exp2f(ml[2 * i] - M);
-        const float *src = ob + (size_t)i * D + lane * DPL;
-#pragma unroll
-        for (int k = 0; k < DPL; ++k) acc[k] = fmaf(w, src[k], acc[k]);
+        den = fmaf(w, ml[2 * i + 1], den);
+        const float *src = ob + (size_t)i * D + lane * VL;
+        if constexpr (VL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(src);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+        }
     }
-    const float inv = 1.f / den;
-    T *dst = static_cast<T *>(p.out) + (size_t)row * D + lane * DPL;
 #pragma unroll
-    for (int k = 0; k < DPL; ++k) dst[k] = Elem<T>::from_float(acc[k] * inv);
+    for (int k = 0; k < VL; ++k) s_acc[warp][lane * VL + k] = acc[k];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+
+    for (int idx = threadIdx.x; idx < D / E; idx += NW * 32) {
+        float dsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) dsum += s_den[w];
+        const float inv = 1.f / dsum;
+        float v[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) t += s_acc[w][idx * E + e];
+            v[e] = t * inv;
+        }
+        store_row<T, E>(static_cast<T *>(p.out) + (size_t)row * D + idx * E, v);
+    }
 }
 
 }  // namespace pkv

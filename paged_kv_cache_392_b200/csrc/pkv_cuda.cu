@@ -79,7 +79,8 @@ pkv_status check_attn_desc(const pkv_attn_desc *d, const char *fn, Split *sp) {
     sp->part_blocks = pt / pkv::kBlock;
     sp->pmax = (d->max_blocks_per_seq + sp->part_blocks - 1) / sp->part_blocks;
     const int64_t grid = (int64_t)d->num_seqs * d->num_kv_heads * sp->pmax;
-    if (grid > INT_MAX) return fail(PKV_ERR_INVALID, "%s: batch too large for one launch", fn);
+    if (grid > INT_MAX || (int64_t)d->num_seqs * d->num_q_heads > INT_MAX)
+        return fail(PKV_ERR_INVALID, "%s: batch too large for one launch", fn);
     return PKV_OK;
 }
 
@@ -147,8 +148,8 @@ pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t str
                                   void (*kern)(const pkv::DecodeParams)) {
     if (prm.pmax <= 1) return PKV_OK;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(((int64_t)prm.S * prm.Hq + 3) / 4));
-    cfg.blockDim = dim3(128);
+    cfg.gridDim = dim3((unsigned)((int64_t)prm.S * prm.Hq));
+    cfg.blockDim = dim3(pkv::kReduceWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -201,21 +202,7 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, cudaStream_t stream) {
     kern<<<grid, kWarps * 32, Cfg::SMEM, stream>>>(prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "decode launch");
-    if (prm.pmax > 1) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(((int64_t)prm.S * prm.Hq + 3) / 4));
-        cfg.blockDim = dim3(128);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, pkv::lse_reduce_kernel<T, D>, prm);
-        if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "reduce launch");
-    }
-    return PKV_OK;
+    return launch_reduce_if_split(prm, stream, pkv::lse_reduce_kernel<T, D>);
 }
 
 // Whether the tensor-core kernel serves this call: 16-bit K/V whose 2-D TMA view fits int32

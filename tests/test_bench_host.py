@@ -1,0 +1,91 @@
+"""CPU checks of bench.py's host logic: the reference (oracle) arm's JSON line, the
+multi-process launch where rank 0 alone reports, and the max-over-ranks timing reduction
+over a world-size-2 gloo group."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+        "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "impl",
+        "cpu_baseline", "e2e"}
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                          "tiny", "--steps", "2", "--warmup", "1"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert KEYS <= set(d)
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] >= 1
+
+
+def test_reference_arm_under_two_ranks_reports_once():
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py",
+           "--impl", "reference", "--workload", "tiny", "--gpus", "2", "--steps", "1",
+           "--warmup", "0"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1 and json.loads(lines[0])["n_gpus"] == 2
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    w, r, lr = bench.dist_env()
+    dist = bench.init_dist(w, backend="gloo")
+    dev = torch.device("cpu")
+    bench.barrier(dist, dev)
+    m = bench.max_over_ranks(dist, 1.5 + rank, dev)
+    bench.barrier(dist, dev)
+    dist.destroy_process_group()
+    q.put((r, w, m))
+
+
+def test_max_over_ranks_with_gloo_world_size_2():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, 2, 2.5), (1, 2, 2.5)]
+
+
+def test_algorithmic_bytes_and_split_rows():
+    from paged_kv_cache_392_b200 import workloads as W
+    wl = W.tiny()
+    import numpy as np
+    nb = bench.algorithmic_bytes(wl, np.zeros((0, 2), np.int32))
+    assert nb["kv"] == (5 + 17 + 33 + 48) * 2 * 64 * 4 * 2
+    assert nb["decode"] > nb["kv"] and nb["kv_copy"] == 0
+    rows, pmax = bench.split_rows(wl, 16)
+    # lengths 5, 17, 33, 48 over 16-token partitions: 1, 2, 3, 3 partitions
+    assert pmax == 3 and rows == (2 + 3 + 3) * 2
