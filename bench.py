@@ -60,6 +60,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--read-probe", action="store_true",
                     help="also measure a read-only streaming ceiling (torch.sum, 2 GiB)")
+    ap.add_argument("--swap-probe", action="store_true",
+                    help="also time swapping the batch's blocks to pinned host memory and "
+                         "back (kv_swap_out / kv_swap_in over PCIe)")
     ap.add_argument("--contiguous", action="store_true",
                     help="place each sequence's blocks contiguously and in order (paged "
                          "kernel over a contiguous layout) instead of shuffled")
@@ -188,13 +191,16 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+DECODE_SOURCES = ("attn_decode.cuh", "attn_decode_tc.cuh", "ptx.cuh", "faults.cuh")
+
+
 def kernel_source_sha():
+    """Hash of the decode kernels' sources (kernels and their launch shape)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in DECODE_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -300,6 +306,35 @@ def barrier(dist, device):
             dist.barrier(device_ids=[device.index])
         else:
             dist.barrier()
+
+
+def swap_probe(torch, B, wl, kp, vp, device, reps=5):
+    """Swap every block of the batch out to pinned host memory and back in, timed with CUDA
+    events; returns GB/s each way (block bytes of K and V / time)."""
+    used = np.unique(wl.block_tables[wl.block_tables >= 0]).astype(np.int32)
+    n = len(used)
+    hk = torch.empty((n,) + tuple(kp.shape[1:]), dtype=kp.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([used, np.arange(n, dtype=np.int32)], 1)).to(device)
+    in_pairs = torch.from_numpy(np.stack([np.arange(n, dtype=np.int32), used], 1)).to(device)
+    nbytes = 2 * n * kp[0].numel() * kp.element_size()
+    res = {}
+    for name, call in (("out", lambda: B.kv_swap_out(out_pairs, kp, vp, hk, hv)),
+                       ("in", lambda: B.kv_swap_in(in_pairs, hk, hv, kp, vp))):
+        call()
+        torch.cuda.synchronize()
+        best = 0.0
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+        res[name + "_gbs"] = round(best, 2)
+    res["bytes"] = nbytes
+    res["blocks"] = n
+    return res
 
 
 def read_probe_gbs(torch, device, gib=2, reps=5):
@@ -549,6 +584,7 @@ def run_pkv(args):
         achieved = nbytes["decode"] / (decode_ms * 1e-3) / 1e9
         traffic = profile_traffic(args.workload)
         probe = read_probe_gbs(torch, device) if args.read_probe else None
+        swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe else None
         result = {
             "metric": METRIC,
             "value": round(kv_gbs, 2),
@@ -604,6 +640,7 @@ def run_pkv(args):
                                           2),
                     "serial_ms_per_step": round(e2e_serial_ms, 5)},
             "gpu_launches": K * launches_per_step,
+            "swap": swap,
             "clocks": sampler.summary(),
         }
         if wl.name == "fork":

@@ -134,6 +134,27 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
                           int32_t num_pairs, void *k_pool, void *v_pool, void *stream);
 
 /*
+ * Swap whole blocks between the device pools and a host pool ("vLLM and PagedAttention: How
+ * Ideas from Operating Systems Accelerated LLM Inference": when memory runs short, whole
+ * sequences are evicted by swapping them to CPU memory).  host_k / host_v are pinned host
+ * buffers of num_host_blocks blocks, [num_host_blocks][H_kv][16][D] dtype each, allocated
+ * so the device can reach them (cudaHostAlloc / cudaMallocHost, or torch pin_memory); other
+ * host memory is rejected with PKV_ERR_INVALID before any launch.  pairs is device int32
+ * [num_pairs][2]:
+ *   kv_swap_out: (device block, host block) -- host block := device block, K and V;
+ *   kv_swap_in:  (host block, device block) -- device block := host block, K and V.
+ * Block ids outside their pool are skipped and set PKV_FAULT_BAD_PAIR.  The copies cross
+ * PCIe from the kernel itself (one launch per call, whatever the number of blocks).
+ * pkv_bm_swap_out / pkv_bm_swap_in produce the pairs.
+ */
+pkv_status kv_swap_out(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
+                       const void *k_pool, const void *v_pool, void *host_k, void *host_v,
+                       int32_t num_host_blocks, void *stream);
+pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
+                      const void *host_k, const void *host_v, int32_t num_host_blocks,
+                      void *k_pool, void *v_pool, void *stream);
+
+/*
  * Allocation-free variant of paged_attn_decode.  The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory -- for example a serving
  * engine that hands (nearly) all free HBM to its KV pool at start-up and owns every later
@@ -225,6 +246,30 @@ int32_t pkv_bm_num_seqs(const pkv_bm *bm);
 
 /* Copy the free list, head first, into out (host, capacity cap); returns its length. */
 int32_t pkv_bm_free_list(const pkv_bm *bm, int32_t *out, int32_t cap);
+
+/* Host (swap) pool of num_host_blocks blocks with its own first-in first-out free list
+ * (initial_free_order: permutation or NULL = ascending).  Host blocks each hold one swapped
+ * sequence's data and are never shared.  Fails while any sequence is swapped out. */
+pkv_status pkv_bm_set_host_pool(pkv_bm *bm, int32_t num_host_blocks,
+                                const int32_t *initial_free_order);
+
+/* Evict seq to the host pool: each table entry j gets a fresh host block h_j and
+ * pairs_out[j] = (device block, h_j) (host, capacity cap pairs; *n = table length).  The
+ * device block loses one reference and returns to the free list when none is left, so run
+ * kv_swap_out on these pairs before any later write can reuse it.  All or nothing
+ * (PKV_ERR_OOM when the host pool is short).  A swapped-out sequence can only be swapped
+ * in or freed. */
+pkv_status pkv_bm_swap_out(pkv_bm *bm, int64_t seq, int32_t *pairs_out, int32_t cap,
+                           int32_t *n);
+
+/* Bring seq back: each host block gets a fresh device block, pairs_out[j] = (host block,
+ * device block); the host blocks return to the host free list.  All or nothing.  Blocks
+ * that were shared before the swap come back as private copies. */
+pkv_status pkv_bm_swap_in(pkv_bm *bm, int64_t seq, int32_t *pairs_out, int32_t cap,
+                          int32_t *n);
+
+pkv_status pkv_bm_is_swapped(const pkv_bm *bm, int64_t seq, int32_t *swapped);
+int32_t pkv_bm_num_host_free(const pkv_bm *bm);
 
 #ifdef __cplusplus
 }

@@ -53,6 +53,8 @@ def lib():
         L.orc_kv_write.restype = i32
         L.orc_kv_copy_blocks.argtypes = [i32, vp] + [i32] * 5 + [vp, vp]
         L.orc_kv_copy_blocks.restype = i32
+        L.orc_kv_swap.argtypes = [i32, vp, vp, vp, i32, vp, vp, i32, ctypes.c_size_t]
+        L.orc_kv_swap.restype = i32
         _lib = L
     return _lib
 
@@ -180,3 +182,18 @@ def kv_copy_blocks(pairs, k_pool, v_pool):
     rc = lib().orc_kv_copy_blocks(pr.shape[0], _ptr(pr), Hkv, D, B, NB,
                                   k_pool.dtype.itemsize, _ptr(k_pool), _ptr(v_pool))
     _check(rc, "kv_copy_blocks")
+
+
+def kv_swap(pairs, src_k, src_v, dst_k, dst_v):
+    """Block dst of (dst_k, dst_v) := block src of (src_k, src_v) for each (src, dst) pair.
+    Pools are [blocks, Hkv, B, D] arrays of one element size (device <-> host swap)."""
+    for a in (src_k, src_v, dst_k, dst_v):
+        if not a.flags.c_contiguous:
+            raise ValueError("arrays must be C-contiguous")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype.itemsize != dst_k.dtype.itemsize:
+        raise ValueError("block shapes differ")
+    bb = int(np.prod(src_k.shape[1:])) * src_k.dtype.itemsize
+    pr = np.ascontiguousarray(pairs, dtype=np.int32).reshape(-1, 2)
+    rc = lib().orc_kv_swap(pr.shape[0], _ptr(pr), _ptr(src_k), _ptr(src_v), src_k.shape[0],
+                           _ptr(dst_k), _ptr(dst_v), dst_k.shape[0], bb)
+    _check(rc, "kv_swap")

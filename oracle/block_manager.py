@@ -15,7 +15,12 @@ Rules, from "Memory Optimization in LLM Serving with PagedAttention":
     reference count, and if it is above one it takes a fresh block, copies the old block's
     content there, repoints its own table entry, and only then writes.
 And from "vLLM and PagedAttention: How Ideas from Operating Systems Accelerated LLM
-Inference": 16-token blocks by default; memory is allocated as generation proceeds.
+Inference": 16-token blocks by default; memory is allocated as generation proceeds; when
+memory runs short, whole sequences are evicted by swapping them to CPU
+memory.  Modelled here as a second, host pool of blocks: swapping a sequence out gives each of
+its blocks a fresh host block (the device block loses one reference and is freed when none is
+left), swapping it in gives each host block a fresh device block; a swapped-out sequence can
+only be swapped in or freed.
 
 Readings where the pages are silent:
   * the free list is first-in first-out: allocation pops its head, a freed block joins its
@@ -46,6 +51,19 @@ class BlockManagerModel:
         self.ref = [0] * num_blocks
         self.tables = {}
         self.lens = {}
+        self.swapped = set()
+        self.host_free = deque()
+        self.num_host_blocks = 0
+
+    def set_host_pool(self, num_host_blocks, free_order=None):
+        order = list(range(num_host_blocks)) if free_order is None else \
+            [int(b) for b in free_order]
+        if sorted(order) != list(range(num_host_blocks)):
+            raise ValueError("host free order must be a permutation")
+        if self.swapped:
+            raise ValueError("sequences are swapped out")
+        self.num_host_blocks = num_host_blocks
+        self.host_free = deque(order)
 
     # -- queries --------------------------------------------------------------------
     def num_free(self):
@@ -62,6 +80,14 @@ class BlockManagerModel:
 
     def free_order(self):
         return list(self.free)
+
+    def host_free_order(self):
+        return list(self.host_free)
+
+    def is_swapped(self, seq):
+        if seq not in self.tables:
+            raise KeyError(seq)
+        return seq in self.swapped
 
     def waste(self, seq):
         """Empty slots in the sequence's own blocks (internal fragmentation)."""
@@ -91,6 +117,8 @@ class BlockManagerModel:
     def append_slot(self, seq):
         """Give the next token of ``seq`` a slot; returns (slot, cow) with cow = (src, dst)
         when a shared last block had to be copied first, else None."""
+        if seq in self.swapped:
+            raise ValueError("sequence is swapped out")
         table = self.tables[seq]
         n = self.lens[seq]
         B = self.block_size
@@ -111,6 +139,8 @@ class BlockManagerModel:
     def append_slots(self, seqs):
         """Append one token to each sequence in order; all or nothing.
         Returns (slots, cow_pairs)."""
+        if any(s in self.swapped for s in seqs):
+            raise ValueError("sequence is swapped out")
         saved = (copy.copy(self.free), list(self.ref),
                  {s: list(t) for s, t in self.tables.items()}, dict(self.lens))
         slots, pairs = [], []
@@ -129,6 +159,8 @@ class BlockManagerModel:
         """``child`` maps the same physical blocks as ``parent`` (shared pages)."""
         if child in self.tables:
             raise KeyError("child exists")
+        if parent in self.swapped:
+            raise ValueError("parent is swapped out")
         table = self.tables[parent]
         for blk in table:
             self.ref[blk] += 1
@@ -137,8 +169,47 @@ class BlockManagerModel:
 
     def free_seq(self, seq):
         """Drop a finished sequence; blocks nobody else maps go back to the free list."""
-        for blk in self.tables.pop(seq):
+        if seq in self.swapped:
+            self.swapped.discard(seq)
+            self.host_free.extend(self.tables.pop(seq))
+        else:
+            for blk in self.tables.pop(seq):
+                self.ref[blk] -= 1
+                if self.ref[blk] == 0:
+                    self.free.append(blk)
+        del self.lens[seq]
+
+    def swap_out(self, seq):
+        """Move ``seq`` to host blocks.  Returns [(device_block, host_block), ...] in table
+        order: the copies the caller must make before any freed device block is reused."""
+        if seq in self.swapped:
+            raise ValueError("already swapped out")
+        table = self.tables[seq]
+        if len(table) > len(self.host_free):
+            raise OutOfBlocks("host pool exhausted")
+        pairs = []
+        for j, blk in enumerate(table):
+            h = self.host_free.popleft()
+            pairs.append((blk, h))
             self.ref[blk] -= 1
             if self.ref[blk] == 0:
                 self.free.append(blk)
-        del self.lens[seq]
+            table[j] = h
+        self.swapped.add(seq)
+        return pairs
+
+    def swap_in(self, seq):
+        """Move ``seq`` back to fresh device blocks.  Returns [(host_block, device_block)]."""
+        if seq not in self.swapped:
+            raise ValueError("not swapped out")
+        table = self.tables[seq]
+        if len(table) > len(self.free):
+            raise OutOfBlocks("no free block")
+        pairs = []
+        for j, h in enumerate(table):
+            blk = self._take()
+            pairs.append((h, blk))
+            self.host_free.append(h)
+            table[j] = blk
+        self.swapped.discard(seq)
+        return pairs

@@ -320,3 +320,24 @@ int orc_kv_copy_blocks(int P, const int32_t *pairs, int Hkv, int D, int B, int N
     }
     return err;
 }
+
+/*
+ * Swap copy between two pools of equal block shape (a device pool and a host pool): for each
+ * pair (src, dst), block dst of the destination pools becomes a byte copy of block src of the
+ * source pools, for K and V.  "vLLM and PagedAttention: How Ideas from Operating Systems
+ * Accelerated LLM Inference": evicted sequences are swapped to CPU memory and back.
+ */
+int orc_kv_swap(int P, const int32_t *pairs, const void *src_k, const void *src_v, int nb_src,
+                void *dst_k, void *dst_v, int nb_dst, size_t block_bytes) {
+    if (P < 0 || nb_src < 0 || nb_dst < 0) return ORC_BAD_ARG;
+    int err = ORC_OK;
+    for (int i = 0; i < P; ++i) {
+        int32_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        if (s < 0 || s >= nb_src || d < 0 || d >= nb_dst) { err = ORC_BAD_BLOCK; continue; }
+        memcpy((char *)dst_k + (size_t)d * block_bytes, (const char *)src_k + (size_t)s * block_bytes,
+               block_bytes);
+        memcpy((char *)dst_v + (size_t)d * block_bytes, (const char *)src_v + (size_t)s * block_bytes,
+               block_bytes);
+    }
+    return err;
+}

@@ -28,6 +28,8 @@ EXPORTS = [
     "pkv_bm_add_seq", "pkv_bm_append_slot", "pkv_bm_append_slots", "pkv_bm_fork",
     "pkv_bm_free_seq", "pkv_bm_block_table", "pkv_bm_block_tables", "pkv_bm_seq_len",
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
+    "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
+    "pkv_bm_is_swapped", "pkv_bm_num_host_free",
 ]
 
 
@@ -85,6 +87,13 @@ def lib():
         "pkv_bm_num_free": ([vp], i32),
         "pkv_bm_num_seqs": ([vp], i32),
         "pkv_bm_free_list": ([vp, vp, i32], i32),
+        "kv_swap_out": ([dp, vp, i32, vp, vp, vp, vp, i32, vp], i32),
+        "kv_swap_in": ([dp, vp, i32, vp, vp, i32, vp, vp, vp], i32),
+        "pkv_bm_set_host_pool": ([vp, i32, vp], i32),
+        "pkv_bm_swap_out": ([vp, i64, vp, i32, P(i32)], i32),
+        "pkv_bm_swap_in": ([vp, i64, vp, i32, P(i32)], i32),
+        "pkv_bm_is_swapped": ([vp, i64, P(i32)], i32),
+        "pkv_bm_num_host_free": ([vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -242,6 +251,39 @@ def kv_copy_blocks(src_dst_pairs, k_pool, v_pool, stream=None):
                                 _stream(stream, k_pool.device)))
 
 
+def _host_pool(t, name, like):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_pinned():
+        raise ValueError("%s must be a pinned host tensor" % name)
+    if not t.is_contiguous() or t.dtype != like.dtype or t.shape[1:] != like.shape[1:]:
+        raise ValueError("%s must be [blocks, H_kv, 16, D] like the pools" % name)
+
+
+def kv_swap_out(pairs, k_pool, v_pool, host_k, host_v, stream=None):
+    """host block h := device block g for each (g, h) row of ``pairs`` (device int32)."""
+    desc = _pool_desc(k_pool, v_pool)
+    _dev(pairs, "pairs", torch.int32)
+    _host_pool(host_k, "host_k", k_pool)
+    _host_pool(host_v, "host_v", k_pool)
+    if host_v.shape != host_k.shape:
+        raise ValueError("host_k and host_v differ")
+    _check(lib().kv_swap_out(ctypes.byref(desc), _ptr(pairs), pairs.shape[0], _ptr(k_pool),
+                             _ptr(v_pool), _ptr(host_k), _ptr(host_v), host_k.shape[0],
+                             _stream(stream, k_pool.device)))
+
+
+def kv_swap_in(pairs, host_k, host_v, k_pool, v_pool, stream=None):
+    """device block g := host block h for each (h, g) row of ``pairs`` (device int32)."""
+    desc = _pool_desc(k_pool, v_pool)
+    _dev(pairs, "pairs", torch.int32)
+    _host_pool(host_k, "host_k", k_pool)
+    _host_pool(host_v, "host_v", k_pool)
+    if host_v.shape != host_k.shape:
+        raise ValueError("host_k and host_v differ")
+    _check(lib().kv_swap_in(ctypes.byref(desc), _ptr(pairs), pairs.shape[0], _ptr(host_k),
+                            _ptr(host_v), host_k.shape[0], _ptr(k_pool), _ptr(v_pool),
+                            _stream(stream, k_pool.device)))
+
+
 def device_faults(clear=True, stream=None, device=None):
     """Synchronise and return the device fault word's set bits as names."""
     word = ctypes.c_uint32(0)
@@ -356,3 +398,36 @@ class BlockManager:
         out = np.empty(max(n, 1), np.int32)
         lib().pkv_bm_free_list(self._h, out.ctypes.data, n)
         return out[:n].tolist()
+
+    # -- host (swap) pool ------------------------------------------------------------------
+    def set_host_pool(self, num_host_blocks, free_order=None):
+        np = self._np
+        order = None
+        if free_order is not None:
+            order = np.ascontiguousarray(free_order, dtype=np.int32)
+        _check(lib().pkv_bm_set_host_pool(self._h, num_host_blocks,
+                                          order.ctypes.data if order is not None else None))
+
+    def _swap(self, fn, seq):
+        np = self._np
+        n = ctypes.c_int32()
+        cap = max(1, len(self.block_table(seq)))
+        out = np.empty((cap, 2), np.int32)
+        _check(fn(self._h, seq, out.ctypes.data, cap, ctypes.byref(n)))
+        return out[:n.value].copy()
+
+    def swap_out(self, seq):
+        """Evict ``seq`` to host blocks; returns int32 [n, 2] (device block, host block)."""
+        return self._swap(lib().pkv_bm_swap_out, seq)
+
+    def swap_in(self, seq):
+        """Bring ``seq`` back; returns int32 [n, 2] (host block, device block)."""
+        return self._swap(lib().pkv_bm_swap_in, seq)
+
+    def is_swapped(self, seq):
+        v = ctypes.c_int32()
+        _check(lib().pkv_bm_is_swapped(self._h, seq, ctypes.byref(v)))
+        return bool(v.value)
+
+    def num_host_free(self):
+        return lib().pkv_bm_num_host_free(self._h)

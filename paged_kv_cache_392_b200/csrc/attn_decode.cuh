@@ -31,6 +31,16 @@
 
 namespace pkv {
 
+// Launch shape of the CUDA-core decode kernel (consumer warps per CTA, stages per warp) and
+// the default context partition; overridable at build time for tuning sweeps.
+#ifndef PKV_DECODE_WARPS
+#define PKV_DECODE_WARPS 4
+#endif
+#ifndef PKV_DECODE_STAGES
+#define PKV_DECODE_STAGES 2
+#endif
+constexpr int kDefaultPartitionTokens = 512;
+
 constexpr int kBlock = 16;                       // tokens per KV block
 constexpr uint64_t kWaitTimeoutNs = 1000000000;  // bounded shared-memory barrier waits (1 s)
 

@@ -25,6 +25,15 @@
 
 #include "attn_decode.cuh"
 
+// Launch shape of the tensor-core decode kernel: 2 warps x 2 stages per CTA measured best
+// (or tied) on every workload; overridable at build time for tuning sweeps.
+#ifndef PKV_DECODE_TC_WARPS
+#define PKV_DECODE_TC_WARPS 2
+#endif
+#ifndef PKV_DECODE_TC_STAGES
+#define PKV_DECODE_TC_STAGES 2
+#endif
+
 namespace pkv {
 
 template <typename T, int D, int G, int W, int NSW>

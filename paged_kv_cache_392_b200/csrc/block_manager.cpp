@@ -19,8 +19,9 @@
 namespace {
 
 struct Seq {
-    std::vector<int32_t> table;
+    std::vector<int32_t> table;  // device block ids, or host block ids while swapped out
     int32_t len = 0;
+    bool swapped = false;
 };
 
 // One append, recorded so that a failed batch can be undone exactly.
@@ -40,6 +41,9 @@ struct pkv_bm {
     std::deque<int32_t> free_list;
     std::vector<int32_t> ref;
     std::unordered_map<int64_t, Seq> seqs;
+    // host (swap) pool: blocks hold one swapped-out sequence's data each, never shared
+    int32_t num_host_blocks = 0;
+    std::deque<int32_t> host_free;
 
     int32_t take() {
         int32_t b = free_list.front();
@@ -159,6 +163,9 @@ pkv_status pkv_bm_append_slot(pkv_bm *bm, int64_t seq, int64_t *slot_out, int32_
     if (it == bm->seqs.end())
         return fail(PKV_ERR_NOT_FOUND, "pkv_bm_append_slot: unknown sequence %lld",
                     (long long)seq);
+    if (it->second.swapped)
+        return fail(PKV_ERR_INVALID, "pkv_bm_append_slot: sequence %lld is swapped out",
+                    (long long)seq);
     Undo u;
     if (!bm->append(seq, it->second, slot_out, cow_src, cow_dst, &u))
         return fail(PKV_ERR_OOM, "pkv_bm_append_slot: no free block");
@@ -170,10 +177,15 @@ pkv_status pkv_bm_append_slots(pkv_bm *bm, const int64_t *seqs, int32_t n, int64
     if (!bm || (n > 0 && (!seqs || !slots_out || !cow_pairs_out)) || !num_cow || n < 0)
         return fail(PKV_ERR_INVALID, "pkv_bm_append_slots: bad argument");
     *num_cow = 0;
-    for (int32_t i = 0; i < n; ++i)
-        if (!bm->seqs.count(seqs[i]))
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seqs[i]);
+        if (it == bm->seqs.end())
             return fail(PKV_ERR_NOT_FOUND, "pkv_bm_append_slots: unknown sequence %lld",
                         (long long)seqs[i]);
+        if (it->second.swapped)
+            return fail(PKV_ERR_INVALID, "pkv_bm_append_slots: sequence %lld is swapped out",
+                        (long long)seqs[i]);
+    }
     std::vector<Undo> log((size_t)n);
     int32_t ncow = 0;
     for (int32_t i = 0; i < n; ++i) {
@@ -199,6 +211,9 @@ pkv_status pkv_bm_fork(pkv_bm *bm, int64_t parent, int64_t child) {
         return fail(PKV_ERR_NOT_FOUND, "pkv_bm_fork: unknown parent %lld", (long long)parent);
     if (bm->seqs.count(child))
         return fail(PKV_ERR_INVALID, "pkv_bm_fork: child %lld exists", (long long)child);
+    if (it->second.swapped)
+        return fail(PKV_ERR_INVALID, "pkv_bm_fork: parent %lld is swapped out",
+                    (long long)parent);
     Seq c = it->second;
     for (int32_t b : c.table) bm->ref[b] += 1;
     bm->seqs.emplace(child, std::move(c));
@@ -211,9 +226,13 @@ pkv_status pkv_bm_free_seq(pkv_bm *bm, int64_t seq) {
     if (it == bm->seqs.end())
         return fail(PKV_ERR_NOT_FOUND, "pkv_bm_free_seq: unknown sequence %lld",
                     (long long)seq);
-    for (int32_t b : it->second.table) {
-        bm->ref[b] -= 1;
-        if (bm->ref[b] == 0) bm->free_list.push_back(b);
+    if (it->second.swapped) {
+        for (int32_t b : it->second.table) bm->host_free.push_back(b);
+    } else {
+        for (int32_t b : it->second.table) {
+            bm->ref[b] -= 1;
+            if (bm->ref[b] == 0) bm->free_list.push_back(b);
+        }
     }
     bm->seqs.erase(it);
     return PKV_OK;
@@ -244,6 +263,9 @@ pkv_status pkv_bm_block_tables(const pkv_bm *bm, const int64_t *seqs, int32_t n,
         if (it == bm->seqs.end())
             return fail(PKV_ERR_NOT_FOUND, "pkv_bm_block_tables: unknown sequence %lld",
                         (long long)seqs[i]);
+        if (it->second.swapped)
+            return fail(PKV_ERR_INVALID, "pkv_bm_block_tables: sequence %lld is swapped out",
+                        (long long)seqs[i]);
         const std::vector<int32_t> &t = it->second.table;
         if ((int64_t)t.size() > max_blocks)
             return fail(PKV_ERR_INVALID, "pkv_bm_block_tables: sequence %lld has %zu blocks > %d",
@@ -270,6 +292,109 @@ pkv_status pkv_bm_refcount(const pkv_bm *bm, int32_t block, int32_t *count) {
         return fail(PKV_ERR_INVALID, "pkv_bm_refcount: block %d out of range", block);
     *count = bm->ref[block];
     return PKV_OK;
+}
+
+pkv_status pkv_bm_set_host_pool(pkv_bm *bm, int32_t num_host_blocks,
+                                const int32_t *initial_free_order) {
+    if (!bm || num_host_blocks < 0)
+        return fail(PKV_ERR_INVALID, "pkv_bm_set_host_pool: bad argument");
+    for (auto &kv : bm->seqs)
+        if (kv.second.swapped)
+            return fail(PKV_ERR_INVALID, "pkv_bm_set_host_pool: sequences are swapped out");
+    std::deque<int32_t> order;
+    if (initial_free_order) {
+        std::vector<char> seen(num_host_blocks, 0);
+        for (int32_t i = 0; i < num_host_blocks; ++i) {
+            int32_t b = initial_free_order[i];
+            if (b < 0 || b >= num_host_blocks || seen[b])
+                return fail(PKV_ERR_INVALID,
+                            "pkv_bm_set_host_pool: initial_free_order is not a permutation");
+            seen[b] = 1;
+            order.push_back(b);
+        }
+    } else {
+        for (int32_t i = 0; i < num_host_blocks; ++i) order.push_back(i);
+    }
+    bm->num_host_blocks = num_host_blocks;
+    bm->host_free.swap(order);
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_swap_out(pkv_bm *bm, int64_t seq, int32_t *pairs_out, int32_t cap,
+                           int32_t *n) {
+    if (!bm || !n || (cap > 0 && !pairs_out))
+        return fail(PKV_ERR_INVALID, "pkv_bm_swap_out: bad argument");
+    *n = 0;
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end())
+        return fail(PKV_ERR_NOT_FOUND, "pkv_bm_swap_out: unknown sequence %lld",
+                    (long long)seq);
+    Seq &s = it->second;
+    if (s.swapped)
+        return fail(PKV_ERR_INVALID, "pkv_bm_swap_out: sequence %lld is already swapped out",
+                    (long long)seq);
+    const int32_t nb = (int32_t)s.table.size();
+    if (cap < nb) return fail(PKV_ERR_INVALID, "pkv_bm_swap_out: capacity %d < %d", cap, nb);
+    if ((size_t)nb > bm->host_free.size())
+        return fail(PKV_ERR_OOM, "pkv_bm_swap_out: need %d host blocks, %zu free", nb,
+                    bm->host_free.size());
+    for (int32_t j = 0; j < nb; ++j) {
+        const int32_t g = s.table[j];
+        const int32_t h = bm->host_free.front();
+        bm->host_free.pop_front();
+        pairs_out[2 * j] = g;
+        pairs_out[2 * j + 1] = h;
+        bm->ref[g] -= 1;
+        if (bm->ref[g] == 0) bm->free_list.push_back(g);
+        s.table[j] = h;
+    }
+    s.swapped = true;
+    *n = nb;
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_swap_in(pkv_bm *bm, int64_t seq, int32_t *pairs_out, int32_t cap,
+                          int32_t *n) {
+    if (!bm || !n || (cap > 0 && !pairs_out))
+        return fail(PKV_ERR_INVALID, "pkv_bm_swap_in: bad argument");
+    *n = 0;
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end())
+        return fail(PKV_ERR_NOT_FOUND, "pkv_bm_swap_in: unknown sequence %lld", (long long)seq);
+    Seq &s = it->second;
+    if (!s.swapped)
+        return fail(PKV_ERR_INVALID, "pkv_bm_swap_in: sequence %lld is not swapped out",
+                    (long long)seq);
+    const int32_t nb = (int32_t)s.table.size();
+    if (cap < nb) return fail(PKV_ERR_INVALID, "pkv_bm_swap_in: capacity %d < %d", cap, nb);
+    if ((size_t)nb > bm->free_list.size())
+        return fail(PKV_ERR_OOM, "pkv_bm_swap_in: need %d blocks, %zu free", nb,
+                    bm->free_list.size());
+    for (int32_t j = 0; j < nb; ++j) {
+        const int32_t h = s.table[j];
+        const int32_t g = bm->take();
+        pairs_out[2 * j] = h;
+        pairs_out[2 * j + 1] = g;
+        bm->host_free.push_back(h);
+        s.table[j] = g;
+    }
+    s.swapped = false;
+    *n = nb;
+    return PKV_OK;
+}
+
+pkv_status pkv_bm_is_swapped(const pkv_bm *bm, int64_t seq, int32_t *swapped) {
+    if (!bm || !swapped) return fail(PKV_ERR_INVALID, "pkv_bm_is_swapped: bad argument");
+    auto it = bm->seqs.find(seq);
+    if (it == bm->seqs.end())
+        return fail(PKV_ERR_NOT_FOUND, "pkv_bm_is_swapped: unknown sequence %lld",
+                    (long long)seq);
+    *swapped = it->second.swapped ? 1 : 0;
+    return PKV_OK;
+}
+
+int32_t pkv_bm_num_host_free(const pkv_bm *bm) {
+    return bm ? (int32_t)bm->host_free.size() : -1;
 }
 
 int32_t pkv_bm_num_free(const pkv_bm *bm) { return bm ? (int32_t)bm->free_list.size() : -1; }

@@ -90,4 +90,44 @@ __global__ void __launch_bounds__(256) kv_copy_blocks_kernel(const KvCopyParams 
     }
 }
 
+// Swap of whole blocks between the device pools and a host pool (pinned, mapped memory
+// reached over PCIe): "vLLM and PagedAttention: How Ideas from Operating Systems Accelerated
+// LLM Inference" -- when memory runs short, whole sequences are evicted to CPU memory and
+// brought back later.  For pair i, block dst of the destination pool becomes a byte copy of
+// block src of the source pool, for K and for V.  One direction per launch.
+struct KvSwapParams {
+    const int32_t *pairs;  // [P][2] (src block, dst block)
+    const uint4 *src_k;
+    const uint4 *src_v;
+    uint4 *dst_k;
+    uint4 *dst_v;
+    int32_t P, nb_src, nb_dst;
+    int64_t vpb;           // 16-byte vectors per block
+};
+
+__global__ void __launch_bounds__(256) kv_swap_kernel(const KvSwapParams p) {
+    const int pair = blockIdx.x >> 1;
+    const int pool = blockIdx.x & 1;
+    const int32_t src = p.pairs[2 * pair];
+    const int32_t dst = p.pairs[2 * pair + 1];
+    if ((unsigned)src >= (unsigned)p.nb_src || (unsigned)dst >= (unsigned)p.nb_dst) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && pool == 0) atomicOr(&g_faults, 0x8u);
+        return;
+    }
+    const uint4 *s = (pool ? p.src_v : p.src_k) + (int64_t)src * p.vpb;
+    uint4 *d = (pool ? p.dst_v : p.dst_k) + (int64_t)dst * p.vpb;
+    const int64_t i0 = (int64_t)blockIdx.y * (kCopyUnroll * 256) + threadIdx.x;
+    uint4 buf[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = i0 + u * 256;
+        if (i < p.vpb) buf[u] = s[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const int64_t i = i0 + u * 256;
+        if (i < p.vpb) d[i] = buf[u];
+    }
+}
+
 }  // namespace pkv

@@ -18,16 +18,10 @@ namespace {
 
 using pkv::fail;
 
-#ifndef PKV_DECODE_WARPS
-#define PKV_DECODE_WARPS 4
-#endif
-#ifndef PKV_DECODE_STAGES
-#define PKV_DECODE_STAGES 2
-#endif
 constexpr int kWarps = PKV_DECODE_WARPS;    // consumer warps per decode CTA
 constexpr int kStages = PKV_DECODE_STAGES;  // shared-memory stages per warp (K+V block each)
 constexpr int kMaxDevices = 64;
-constexpr int kDefaultPartitionTokens = 512;
+constexpr int kDefaultPartitionTokens = pkv::kDefaultPartitionTokens;
 
 int elem_size(int32_t dtype) {
     return dtype == PKV_F32 ? 4 : (dtype == PKV_F16 || dtype == PKV_BF16) ? 2 : 0;
@@ -161,12 +155,6 @@ pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t str
     return cuda_check(e, "paged_attn_decode", "reduce launch");
 }
 
-#ifndef PKV_DECODE_TC_WARPS
-#define PKV_DECODE_TC_WARPS 2
-#endif
-#ifndef PKV_DECODE_TC_STAGES
-#define PKV_DECODE_TC_STAGES 2
-#endif
 constexpr int kTcWarps = PKV_DECODE_TC_WARPS;
 constexpr int kTcStages = PKV_DECODE_TC_STAGES;
 
@@ -438,6 +426,96 @@ pkv_status paged_attn_decode_no_alloc(const pkv_attn_desc *desc, const void *q,
     }
     return paged_attn_decode(desc, q, k_pool, v_pool, block_tables, context_lens, scale, out,
                              ws, need ? (size_t)PKV_STATIC_WORKSPACE_BYTES : 0, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Device-side address of a caller's pinned host buffer; rejects memory the GPU cannot reach.
+pkv_status mapped_host(const void *host, void **dev, const char *fn, const char *name) {
+    cudaPointerAttributes a;
+    cudaError_t e = cudaPointerGetAttributes(&a, host);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(PKV_ERR_INVALID, "%s: %s is not a CUDA-registered host buffer", fn, name);
+    }
+    if (a.type != cudaMemoryTypeHost || !a.devicePointer)
+        return fail(PKV_ERR_INVALID, "%s: %s must be pinned host memory mapped for the device",
+                    fn, name);
+    if (!aligned(a.devicePointer, 16))
+        return fail(PKV_ERR_INVALID, "%s: %s must be 16-byte aligned", fn, name);
+    *dev = a.devicePointer;
+    return PKV_OK;
+}
+
+pkv_status launch_swap(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n,
+                       const void *src_k, const void *src_v, int32_t nb_src, void *dst_k,
+                       void *dst_v, int32_t nb_dst, cudaStream_t stream, const char *fn) {
+    if (n > INT_MAX / 2) return fail(PKV_ERR_INVALID, "%s: too many pairs", fn);
+    pkv::KvSwapParams prm;
+    prm.pairs = pairs;
+    prm.src_k = static_cast<const uint4 *>(src_k);
+    prm.src_v = static_cast<const uint4 *>(src_v);
+    prm.dst_k = static_cast<uint4 *>(dst_k);
+    prm.dst_v = static_cast<uint4 *>(dst_v);
+    prm.P = n;
+    prm.nb_src = nb_src;
+    prm.nb_dst = nb_dst;
+    prm.vpb = (int64_t)desc->num_kv_heads * pkv::kBlock * desc->head_dim *
+              elem_size(desc->dtype) / 16;
+    const int64_t slices = (prm.vpb + pkv::kCopyUnroll * 256 - 1) / (pkv::kCopyUnroll * 256);
+    if (slices > 65535) return fail(PKV_ERR_UNSUPPORTED, "%s: block too large", fn);
+    dim3 grid((unsigned)(2 * n), (unsigned)slices);
+    pkv::kv_swap_kernel<<<grid, 256, 0, stream>>>(prm);
+    return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+pkv_status check_swap_args(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n,
+                           const void *k_pool, const void *v_pool, const void *host_k,
+                           const void *host_v, int32_t num_host_blocks, const char *fn) {
+    pkv_status st = check_pool_desc(desc, fn);
+    if (st) return st;
+    if (n < 0 || num_host_blocks < 0) return fail(PKV_ERR_INVALID, "%s: negative size", fn);
+    if (n > 0 && (!pairs || !k_pool || !v_pool || !host_k || !host_v))
+        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
+    if (n > 0 && (!aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(pairs, 4)))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status kv_swap_out(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
+                       const void *k_pool, const void *v_pool, void *host_k, void *host_v,
+                       int32_t num_host_blocks, void *stream) {
+    const char *fn = "kv_swap_out";
+    pkv_status st = check_swap_args(desc, pairs, num_pairs, k_pool, v_pool, host_k, host_v,
+                                    num_host_blocks, fn);
+    if (st || num_pairs == 0) return st;
+    void *dk = nullptr, *dv = nullptr;
+    if ((st = mapped_host(host_k, &dk, fn, "host_k")) || (st = mapped_host(host_v, &dv, fn,
+                                                                              "host_v")))
+        return st;
+    return launch_swap(desc, pairs, num_pairs, k_pool, v_pool, desc->num_blocks, dk, dv,
+                       num_host_blocks, static_cast<cudaStream_t>(stream), fn);
+}
+
+pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
+                      const void *host_k, const void *host_v, int32_t num_host_blocks,
+                      void *k_pool, void *v_pool, void *stream) {
+    const char *fn = "kv_swap_in";
+    pkv_status st = check_swap_args(desc, pairs, num_pairs, k_pool, v_pool, host_k, host_v,
+                                    num_host_blocks, fn);
+    if (st || num_pairs == 0) return st;
+    void *dk = nullptr, *dv = nullptr;
+    if ((st = mapped_host(host_k, &dk, fn, "host_k")) || (st = mapped_host(host_v, &dv, fn,
+                                                                              "host_v")))
+        return st;
+    return launch_swap(desc, pairs, num_pairs, dk, dv, num_host_blocks, k_pool, v_pool,
+                       desc->num_blocks, static_cast<cudaStream_t>(stream), fn);
 }
 
 pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream) {

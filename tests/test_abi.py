@@ -18,8 +18,7 @@ def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
-    return sorted({n for n in names if n.startswith(("pkv_", "paged_attn_decode")) or n in (
-        "kv_write", "kv_copy_blocks")})
+    return sorted({n for n in names if n.startswith(("pkv_", "paged_attn_decode", "kv_"))})
 
 
 @pytest.fixture(scope="module")
@@ -116,3 +115,15 @@ def test_kv_ops_reject_bad_arguments(lib):
     assert lib.kv_copy_blocks(ctypes.byref(d), None, 2, a, a, None) == 1
     assert lib.kv_copy_blocks(ctypes.byref(_desc(head_dim=80)), a, 2, a, a, None) == 3
     assert lib.pkv_device_faults(None, 0, None) == 1
+
+
+def test_swap_rejects_host_memory_the_device_cannot_reach(lib):
+    import numpy as np
+    d = _desc()
+    a = ctypes.c_void_p(1 << 20)
+    plain = np.zeros(64, np.uint8)          # pageable host memory: never handed to a kernel
+    rc = lib.kv_swap_out(ctypes.byref(d), a, 1, a, a, ctypes.c_void_p(plain.ctypes.data),
+                         ctypes.c_void_p(plain.ctypes.data), 4, None)
+    assert rc in (1, 4) and B.last_error()
+    assert lib.kv_swap_in(ctypes.byref(d), a, -1, a, a, 4, a, a, None) == 1
+    assert lib.kv_swap_out(ctypes.byref(d), None, 0, None, None, None, None, 0, None) == 0

@@ -156,3 +156,93 @@ def test_packed_tables():
     assert t.tolist() == [[2, 3, 4, -1], [0, 1, -1, -1]] and lens.tolist() == [40, 20]
     with pytest.raises(B.PkvError):
         bm.block_tables([6], 2)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_swap_traffic_matches_model(seed):
+    """Swap-out / swap-in mixed with appends, forks and frees: bit-exact with the model."""
+    rng = np.random.default_rng(100 + seed)
+    NB, NH = 40, 30
+    order, horder = rng.permutation(NB), rng.permutation(NH)
+    bm = B.BlockManager(NB, free_order=order)
+    bm.set_host_pool(NH, horder)
+    model = BlockManagerModel(NB, free_order=order)
+    model.set_host_pool(NH, horder)
+    live, nxt = [], 0
+    for _ in range(1500):
+        op = int(rng.integers(0, 10))
+        on_gpu = [s for s in live if not model.is_swapped(s)]
+        swapped = [s for s in live if model.is_swapped(s)]
+        if op == 0 or not live:
+            act = "add"
+        elif op == 1 and on_gpu:
+            act = "fork"
+        elif op == 2:
+            act = "free"
+        elif op == 3 and on_gpu:
+            act = "out"
+        elif op == 4 and swapped:
+            act = "in"
+        elif on_gpu:
+            act = "append"
+        else:
+            act = "none"
+        try:
+            if act == "add":
+                n = int(rng.integers(0, 60))
+                model.add_seq(nxt, n)
+                bm.add_seq(nxt, n)
+                live.append(nxt)
+                nxt += 1
+            elif act == "fork":
+                p = on_gpu[int(rng.integers(len(on_gpu)))]
+                model.fork(p, nxt)
+                bm.fork(p, nxt)
+                live.append(nxt)
+                nxt += 1
+            elif act == "free":
+                s = live.pop(int(rng.integers(len(live))))
+                model.free_seq(s)
+                bm.free_seq(s)
+            elif act == "out":
+                s = on_gpu[int(rng.integers(len(on_gpu)))]
+                pairs = model.swap_out(s)
+                assert [tuple(x) for x in bm.swap_out(s).tolist()] == pairs
+            elif act == "in":
+                s = swapped[int(rng.integers(len(swapped)))]
+                pairs = model.swap_in(s)
+                assert [tuple(x) for x in bm.swap_in(s).tolist()] == pairs
+            elif act == "append":
+                s = on_gpu[int(rng.integers(len(on_gpu)))]
+                m = model.append_slot(s)
+                assert bm.append_slot(s) == m
+        except ModelOOM:
+            # the product must refuse the same operation and stay unchanged
+            call = {"add": lambda: bm.add_seq(nxt, n), "out": lambda: bm.swap_out(s),
+                    "in": lambda: bm.swap_in(s), "append": lambda: bm.append_slot(s)}[act]
+            with pytest.raises(B.OutOfBlocks):
+                call()
+            if live:
+                s = live.pop(0)
+                model.free_seq(s)
+                bm.free_seq(s)
+        assert bm.num_host_free() == len(model.host_free)
+        same_state(bm, model, [s for s in live if not model.is_swapped(s)])
+        for s in live:
+            assert bm.is_swapped(s) == model.is_swapped(s)
+
+
+def test_swapped_sequences_refuse_use():
+    bm = B.BlockManager(8)
+    bm.set_host_pool(8)
+    bm.add_seq(1, 20)
+    bm.swap_out(1)
+    for call in (lambda: bm.append_slot(1), lambda: bm.fork(1, 2),
+                 lambda: bm.block_tables([1], 4), lambda: bm.swap_out(1)):
+        with pytest.raises(B.PkvError):
+            call()
+    assert bm.swap_in(1).shape == (2, 2)
+    with pytest.raises(B.PkvError):
+        bm.swap_in(1)
+    bm.free_seq(1)
+    assert bm.num_free() == 8 and bm.num_host_free() == 8

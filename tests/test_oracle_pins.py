@@ -339,3 +339,19 @@ def test_kv_copy_blocks_copies_whole_blocks():
     assert np.array_equal(kp, exp_k) and np.array_equal(vp, exp_v)
     with pytest.raises(oracle.OracleError):
         oracle.kv_copy_blocks(np.array([[1, 8]], np.int32), kp, vp)
+
+
+def test_kv_swap_copies_blocks_between_pools():
+    rng = np.random.default_rng(44)
+    dk = rng.standard_normal((6, 2, 16, 8)).astype(np.float32)
+    dv = rng.standard_normal((6, 2, 16, 8)).astype(np.float32)
+    hk = np.zeros((4, 2, 16, 8), np.float32)
+    hv = np.zeros((4, 2, 16, 8), np.float32)
+    pairs = np.array([[5, 0], [1, 3]], np.int32)
+    oracle.kv_swap(pairs, dk, dv, hk, hv)
+    ek, ev = np.zeros_like(hk), np.zeros_like(hv)
+    ek[[0, 3]] = dk[[5, 1]]
+    ev[[0, 3]] = dv[[5, 1]]
+    assert np.array_equal(hk, ek) and np.array_equal(hv, ev)
+    with pytest.raises(oracle.OracleError):
+        oracle.kv_swap(np.array([[0, 4]], np.int32), dk, dv, hk, hv)
