@@ -43,6 +43,12 @@ WORKLOAD_TEXT = {
            "sequence",
     "long": "long-context split decode: 8 seqs x 32768 tokens, 32 q / 8 kv heads, head_dim 128, "
             "bf16 KV, block 16, fully shuffled blocks, 512-token partitions + LSE reduce",
+    "beam": "beam search: 16 requests x width 4, 500-token prompts, 64 generated tokens with "
+            "seeded parent selection each step (forks, frees, copy-on-write), then one decode "
+            "step over the 64 beams; fp16, 40 heads MHA, head_dim 128, block 16",
+    "prefix": "shared system prompt: 64 requests forked from one 1000-token prefix, each "
+              "appending its own 64..512-token prompt, then one decode step; bf16, 32 q / 8 "
+              "kv heads, head_dim 128, block 16",
     "fork": "parallel-sampling fork: 16 prompts x 8 samples sharing 1025 prefilled tokens, first "
             "decode step (112 copy-on-write block copies, 128 kv_writes, decode over 1026 "
             "tokens), fp16, 32 heads MHA, head_dim 128, block 16",
@@ -72,10 +78,101 @@ def parse_args(argv=None):
 
 
 # ---- workload construction ---------------------------------------------------------------
+def _new_bm(model_block_manager, NB, rng):
+    if model_block_manager:
+        from oracle.block_manager import BlockManagerModel
+        return _ModelAdapter(BlockManagerModel(NB, free_order=rng.permutation(NB)))
+    from paged_kv_cache_392_b200 import binding as B
+    return B.BlockManager(NB, free_order=rng.permutation(NB))
+
+
+def _beam_search(bm, rng, n_req=16, width=4, prompt=500, steps=64):
+    """Each step every beam appends one token, then each request keeps `width` survivors
+    drawn (with replacement) from its beams; survivors are forks, the old beams are freed."""
+    beams, nxt = [], 0
+    for r in range(n_req):
+        bm.add_seq(nxt, prompt)
+        group = [nxt]
+        nxt += 1
+        for _ in range(1, width):
+            bm.fork(group[0], nxt)
+            group.append(nxt)
+            nxt += 1
+        beams.append(group)
+    copies = 0
+    for _ in range(steps):
+        _, pairs = bm.append_slots([b for g in beams for b in g])
+        copies += len(pairs)
+        for r in range(n_req):
+            parents = rng.integers(0, width, size=width)
+            new = []
+            for pi in parents:
+                bm.fork(beams[r][int(pi)], nxt)
+                new.append(nxt)
+                nxt += 1
+            for b in beams[r]:
+                bm.free_seq(b)
+            beams[r] = new
+    return [b for g in beams for b in g], copies
+
+
+def _shared_prefix(bm, rng, n_req=64, prefix=1000, lo=64, hi=512):
+    """Requests forked from one cached prefix sequence, each appending its own prompt."""
+    tmpl = 1 << 40
+    bm.add_seq(tmpl, prefix)
+    reqs = list(range(n_req))
+    for r in reqs:
+        bm.fork(tmpl, r)
+    user = rng.integers(lo, hi, size=n_req, endpoint=True)
+    copies = 0
+    for t in range(int(user.max())):
+        active = [r for r in reqs if user[r] > t]
+        _, pairs = bm.append_slots(active)
+        copies += len(pairs)
+    return reqs, copies
+
+
+def _sharing_workload(name, model_block_manager):
+    from paged_kv_cache_392_b200 import workloads as W
+    if name == "beam":
+        Hq = Hkv = 40
+        dtype, seed = "f16", 5
+        NB = 2600
+    else:
+        Hq, Hkv = 32, 8
+        dtype, seed = "bf16", 6
+        NB = 6400
+    rng = np.random.default_rng(seed)
+    bm = _new_bm(model_block_manager, NB, rng)
+    if name == "beam":
+        seqs, copies = _beam_search(bm, rng)
+    else:
+        seqs, copies = _shared_prefix(bm, rng)
+    slots, pairs = bm.append_slots(seqs)          # the decode step's own new token
+    bt, lens = bm.block_tables(seqs, 256)
+    maxB = int((bt >= 0).sum(axis=1).max())
+    bt = np.ascontiguousarray(bt[:, :maxB])
+    in_use = NB - bm.num_free()
+    private = int(((lens.astype(np.int64) + 15) // 16).sum())
+    wl = W.Workload(name=name, num_seqs=len(seqs), num_q_heads=Hq, num_kv_heads=Hkv,
+                    head_dim=128, dtype=dtype, context_lens=lens, block_tables=bt,
+                    num_blocks=NB, free_order=np.asarray(bm.free_order(), np.int32),
+                    slot_mapping=np.asarray(slots, np.int64), scale=1.0 / math.sqrt(128),
+                    seed=seed)
+    wl.extra["unique_blocks"] = in_use
+    wl.extra["sharing"] = {"blocks_in_use": in_use, "blocks_without_sharing": private,
+                           "saving": round(1.0 - in_use / private, 4),
+                           "copy_on_write_copies_before_step": copies}
+    bm.close()
+    return wl, np.asarray(pairs, np.int32).reshape(-1, 2)
+
+
 def build_workload(name, model_block_manager=False):
     """Return (Workload, cow_pairs int32 [P, 2]).  The fork workload's tables come from a
     block manager: the product's C++ one, or the oracle's Python model for the CPU arm."""
     from paged_kv_cache_392_b200 import workloads as W
+    if name in ("beam", "prefix"):
+        return _sharing_workload(name, model_block_manager)
     if name != "fork":
         return W.CONFIGS[name](), np.zeros((0, 2), np.int32)
     f = W.FORK
@@ -118,6 +215,9 @@ class _ModelAdapter:
 
     def fork(self, p, c):
         self.m.fork(p, c)
+
+    def free_seq(self, s):
+        self.m.free_seq(s)
 
     def append_slots(self, seqs):
         slots, pairs = self.m.append_slots(seqs)
@@ -377,8 +477,8 @@ def run_pkv(args):
 
     wl, pairs = build_workload(args.workload)
     if args.contiguous:
-        if args.workload == "fork":
-            raise SystemExit("--contiguous does not apply to the fork workload")
+        if args.workload in ("fork", "beam", "prefix"):
+            raise SystemExit("--contiguous does not apply to the sharing workloads")
         contiguous_placement(wl)
     pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens
     vals = W.make_values(wl, device)
@@ -643,11 +743,13 @@ def run_pkv(args):
             "swap": swap,
             "clocks": sampler.summary(),
         }
-        if wl.name == "fork":
+        if "unique_blocks" in wl.extra:
             uniq = wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim * \
                 wl.elem_size * 2
             result["config"]["unique_kv_bytes"] = uniq
             result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
+        if "sharing" in wl.extra:
+            result["sharing"] = wl.extra["sharing"]
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(wl, vals, args.cpu_seconds)
     if dist is not None:

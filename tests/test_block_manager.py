@@ -246,3 +246,21 @@ def test_swapped_sequences_refuse_use():
         bm.swap_in(1)
     bm.free_seq(1)
     assert bm.num_free() == 8 and bm.num_host_free() == 8
+
+
+@pytest.mark.parametrize("name", ["beam", "prefix"])
+def test_sharing_workloads_match_model(name):
+    """Beam search and shared-prefix traffic: the product manager and the model build the
+    same tables, slots and copy-on-write pairs; sharing saves blocks."""
+    import bench
+    wl, pairs = bench.build_workload(name)
+    wl2, pairs2 = bench.build_workload(name, model_block_manager=True)
+    assert np.array_equal(wl.block_tables, wl2.block_tables)
+    assert np.array_equal(wl.slot_mapping, wl2.slot_mapping)
+    assert np.array_equal(wl.context_lens, wl2.context_lens)
+    assert np.array_equal(pairs, pairs2)
+    sh = wl.extra["sharing"]
+    assert sh == wl2.extra["sharing"]
+    assert 0.3 < sh["saving"] < 0.95
+    if name == "beam":
+        assert len(pairs) > 0        # the decode step's token lands in shared partial blocks

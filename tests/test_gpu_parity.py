@@ -269,3 +269,43 @@ def test_bad_device_values_set_fault_bits_and_touch_nothing_else():
     B.kv_copy_blocks(torch.tensor([[0, wl.num_blocks]], dtype=torch.int32, device="cuda"),
                      vals["k_pool"], vals["v_pool"])
     assert B.device_faults() == ["bad copy pair"]
+
+
+@pytest.mark.parametrize("name", ["beam", "prefix"])
+def test_sharing_workloads_decode_step(name):
+    """One decode step of the beam-search / shared-prefix workloads (tables from the product
+    block manager): copy-on-write copies, kv_write, decode, against the oracle; and the same
+    step over private copies of every block is bit-identical."""
+    import bench
+    wl, pairs = bench.build_workload(name)
+    d = W.make_values(wl, "cuda")
+    kp, vp = bits(d["k_pool"]).copy(), bits(d["v_pool"]).copy()    # before the step
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    B.kv_copy_blocks(torch.from_numpy(pairs).cuda(), d["k_pool"], d["v_pool"])
+    B.kv_write(d["k_new"], d["v_new"], torch.from_numpy(wl.slot_mapping).cuda(), d["k_pool"],
+               d["v_pool"])
+    out = B.paged_attn_decode(d["q"], d["k_pool"], d["v_pool"], bt, lens, wl.scale)
+    torch.cuda.synchronize()
+    oracle.kv_copy_blocks(pairs, kp, vp)
+    oracle.kv_write(bits(d["k_new"]), bits(d["v_new"]), wl.slot_mapping, kp, vp)
+    assert np.array_equal(bits(d["k_pool"]), kp) and np.array_equal(bits(d["v_pool"]), vp)
+    rows = _sample_rows(wl, 32, 1)
+    got = as_f64(out)[rows[:, 0], rows[:, 1]]
+    ref = oracle.paged_attn_decode(bits(d["q"]), kp, vp, wl.block_tables, wl.context_lens,
+                                   wl.scale, wl.dtype, rows=rows)
+    assert np.max(np.abs(got - ref)) <= TOL[wl.dtype]
+    # private layout: gather every sequence's blocks into its own fresh blocks
+    nb = (wl.context_lens + 15) // 16
+    total = int(nb.sum())
+    src = np.concatenate([wl.block_tables[i, :nb[i]] for i in range(wl.num_seqs)])
+    kp2 = d["k_pool"][torch.from_numpy(src).long().cuda()].contiguous()
+    vp2 = d["v_pool"][torch.from_numpy(src).long().cuda()].contiguous()
+    bt2 = np.full_like(wl.block_tables, -1)
+    off = 0
+    for i in range(wl.num_seqs):
+        bt2[i, :nb[i]] = np.arange(off, off + nb[i])
+        off += nb[i]
+    assert off == total
+    out2 = B.paged_attn_decode(d["q"], kp2, vp2, torch.from_numpy(bt2).cuda(), lens, wl.scale)
+    assert torch.equal(out, out2)
