@@ -66,6 +66,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--read-probe", action="store_true",
                     help="also measure a read-only streaming ceiling (torch.sum, 2 GiB)")
+    ap.add_argument("--kv-fp8", action="store_true",
+                    help="FP8 (E4M3) KV cache: kv_write_fp8 + paged_attn_decode_fp8 "
+                         "(opt13b, gqa, long)")
     ap.add_argument("--swap-probe", action="store_true",
                     help="also time swapping the batch's blocks to pinned host memory and "
                          "back (kv_swap_out / kv_swap_in over PCIe)")
@@ -256,18 +259,20 @@ def contiguous_placement(wl):
     wl.extra["placement"] = "contiguous"
 
 
-def algorithmic_bytes(wl, pairs, split_rows=0, pmax_used=None):
-    """Bytes one step must move, counted from the definition of each kernel's work."""
+def algorithmic_bytes(wl, pairs, split_rows=0, kv_es=None):
+    """Bytes one step must move, counted from the definition of each kernel's work.
+    kv_es: bytes per cached K/V element (default the workload dtype's; 1 for FP8)."""
     es = wl.elem_size
+    kv_es = kv_es or es
     S, Hq, Hkv, D = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
-    kv = wl.kv_bytes()                                    # K and V of every cached token
+    kv = int(wl.context_lens.astype(np.int64).sum()) * Hkv * D * kv_es * 2  # K and V once
     qo = S * Hq * D * es * 2                              # q read + out written
     tables = int(((wl.context_lens + 15) // 16).sum()) * 4 + S * 4
     ws = 0
     if split_rows:                                        # partials written + read
         ws = split_rows * (D + 2) * 4 * 2
-    write = S * Hkv * D * es * 2 * 2 + S * 8              # kv_write: read new + write pool
-    copy = len(pairs) * Hkv * 16 * D * es * 2 * 2         # each pair: read + write K and V
+    write = S * Hkv * D * (es + kv_es) * 2 + S * 8        # kv_write: read new + write pool
+    copy = len(pairs) * Hkv * 16 * D * kv_es * 2 * 2      # each pair: read + write K and V
     return {"kv": kv, "decode": kv + qo + tables + ws, "kv_write": write, "kv_copy": copy,
             "step": kv + qo + tables + ws + write + copy}
 
@@ -481,26 +486,44 @@ def run_pkv(args):
             raise SystemExit("--contiguous does not apply to the sharing workloads")
         contiguous_placement(wl)
     pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens
-    vals = W.make_values(wl, device)
+    fp8 = args.kv_fp8
+    if fp8 and (args.workload not in ("opt13b", "gqa", "long") or wl.head_dim != 128):
+        raise SystemExit("--kv-fp8 applies to the opt13b, gqa and long workloads")
+    vals = W.make_values_fp8(wl, device) if fp8 else W.make_values(wl, device)
     q, kp, vp, kn, vn = (vals[k] for k in ("q", "k_pool", "v_pool", "k_new", "v_new"))
+    ksc, vsc = vals.get("k_scale"), vals.get("v_scale")
     bt = torch.from_numpy(wl.block_tables).to(device)
     lens = torch.from_numpy(wl.context_lens).to(device)
     slots = torch.from_numpy(np.ascontiguousarray(wl.slot_mapping, np.int64)).to(device)
     pairs_d = torch.from_numpy(np.ascontiguousarray(pairs, np.int32)).to(device)
     out = torch.empty_like(q)
-    desc = B.decode_desc(q, kp, vp, bt, pt)
+    desc = B.make_desc(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                       wl.num_blocks, bt.shape[1], q.dtype, pt or 0)
     ws_bytes = B.attn_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     npairs = len(pairs)
     rows_split, pmax = split_rows(wl, pt)
-    nbytes = algorithmic_bytes(wl, pairs, rows_split)
+    nbytes = algorithmic_bytes(wl, pairs, rows_split, kv_es=1 if fp8 else None)
+
+    def write(kn_, vn_, slots_):
+        if fp8:
+            B.kv_write_fp8(kn_, vn_, slots_, ksc, vsc, kp, vp)
+        else:
+            B.kv_write(kn_, vn_, slots_, kp, vp)
+
+    def decode(q_, bt_, lens_, out_):
+        if fp8:
+            B.paged_attn_decode_fp8(q_, kp, vp, ksc, vsc, bt_, lens_, wl.scale, out=out_,
+                                    workspace=ws, partition_tokens=pt)
+        else:
+            B.paged_attn_decode(q_, kp, vp, bt_, lens_, wl.scale, out=out_, workspace=ws,
+                                partition_tokens=pt)
 
     def step():
         if npairs:
             B.kv_copy_blocks(pairs_d, kp, vp)
-        B.kv_write(kn, vn, slots, kp, vp)
-        B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
-                            partition_tokens=pt)
+        write(kn, vn, slots)
+        decode(q, bt, lens, out)
 
     launches_per_step = (1 if npairs else 0) + 1 + 1 + (1 if pmax > 1 else 0)
 
@@ -527,10 +550,9 @@ def run_pkv(args):
             for j in range(nsteps):
                 if npairs:
                     B.kv_copy_blocks(pairs_d, kp, vp)
-                B.kv_write(kn, vn, slots, kp, vp)
+                write(kn, vn, slots)
                 ev[j][0].record(gs)
-                B.paged_attn_decode(q, kp, vp, bt, lens, wl.scale, out=out, workspace=ws,
-                                    partition_tokens=pt)
+                decode(q, bt, lens, out)
                 ev[j][1].record(gs)
         return g
 
@@ -587,9 +609,8 @@ def run_pkv(args):
         d = bufs[b]
         if npairs:
             B.kv_copy_blocks(d["pairs"], kp, vp)
-        B.kv_write(d["kn"], d["vn"], d["slots"], kp, vp)
-        B.paged_attn_decode(d["q"], kp, vp, d["bt"], d["lens"], wl.scale, out=outs[b],
-                            workspace=ws, partition_tokens=pt)
+        write(d["kn"], d["vn"], d["slots"])
+        decode(d["q"], d["bt"], d["lens"], outs[b])
 
     def h2d_copy(b, stream):
         with torch.cuda.stream(stream):
@@ -682,9 +703,9 @@ def run_pkv(args):
         step_ms = ms / K
         kv_gbs = world * nbytes["kv"] / (step_ms * 1e-3) / 1e9
         achieved = nbytes["decode"] / (decode_ms * 1e-3) / 1e9
-        traffic = profile_traffic(args.workload)
+        traffic = None if fp8 else profile_traffic(args.workload)
         probe = read_probe_gbs(torch, device) if args.read_probe else None
-        swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe else None
+        swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe and not fp8 else None
         result = {
             "metric": METRIC,
             "value": round(kv_gbs, 2),
@@ -696,7 +717,9 @@ def run_pkv(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32 accumulate over %s KV" % wl.dtype,
+            "dtype": ("f32 accumulate over fp8-e4m3 KV (codes widened to f16 for the "
+                      "tensor-core tiles), %s q/out" % wl.dtype) if fp8 else
+                     "f32 accumulate over %s KV" % wl.dtype,
             "data": "synthetic (seeded), no weights",
             "seqs_per_s": round(world * wl.num_seqs / (step_ms * 1e-3), 1),
             "hbm_frac_step": round(kv_gbs / world / peak, 4),
@@ -705,7 +728,7 @@ def run_pkv(args):
                 "name": args.workload,
                 "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
                 "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-                "block_size": 16, "kv_dtype": wl.dtype,
+                "block_size": 16, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
                 "context_tokens": int(wl.context_lens.sum()),
                 "partition_tokens": pt or 512, "cow_pairs_per_step": npairs,
                 "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
@@ -716,7 +739,7 @@ def run_pkv(args):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "paged_attn_decode (decode + lse_reduce)",
+                "kernel": "paged_attn_decode%s (decode + lse_reduce)" % ("_fp8" if fp8 else ""),
                 "achieved": round(achieved, 1),
                 "peak": peak,
                 "peak_kind": peak_kind,
@@ -750,7 +773,7 @@ def run_pkv(args):
             result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
         if "sharing" in wl.extra:
             result["sharing"] = wl.extra["sharing"]
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and not fp8:
             result["cpu_baseline"] = cpu_baseline(wl, vals, args.cpu_seconds)
     if dist is not None:
         barrier(dist, device)

@@ -45,7 +45,9 @@ typedef enum pkv_status {
     PKV_ERR_NOT_FOUND = 5     /* block manager: unknown sequence id                     */
 } pkv_status;
 
-typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2 } pkv_dtype;
+/* PKV_FP8_E4M3 names FP8 pools in kv_copy_blocks / kv_swap_* (1-byte elements); the FP8
+ * decode and write take the q / new-value dtype in desc->dtype instead. */
+typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_FP8_E4M3 = 3 } pkv_dtype;
 
 /* Bits of the device fault word. */
 #define PKV_FAULT_BAD_LEN   0x1u  /* context_lens[s] outside [1, max_blocks_per_seq*16]  */
@@ -153,6 +155,35 @@ pkv_status kv_swap_out(const pkv_attn_desc *desc, const int32_t *pairs, int32_t 
 pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
                       const void *host_k, const void *host_v, int32_t num_host_blocks,
                       void *k_pool, void *v_pool, void *stream);
+
+/*
+ * FP8 (E4M3) KV cache ("Memory Optimization in LLM Serving with PagedAttention", section
+ * "Broader Context: vLLM, TGI, and TensorRT-LLM": paged KV caches also kept in INT8/FP8).
+ * Format (this library's; the page names none):
+ *   - k_scale, v_scale: device fp32 [H_kv]; element x is stored as the E4M3 code of
+ *     x / scale (fp32 division, round to nearest even, saturating to +-448) and means
+ *     code * scale;
+ *   - k_pool: [NB][H_kv][16][D] bytes;  v_pool: [NB][H_kv][D][16] bytes, transposed, where
+ *     slot p of a row holds token 2*(p>>2) + (p&1) + 8*((p>>1)&1) of the block.
+ * Only head_dim 128 is built.  Pools are 16-byte aligned.  kv_copy_blocks and kv_swap_* move
+ * these blocks with desc->dtype = PKV_FP8_E4M3.
+ *
+ * kv_write_fp8: desc->dtype is the type of k_new / v_new ([T][H_kv][D]); codes are written
+ * into the slots of slot_mapping (-1 skips; others range-checked on the device).
+ *
+ * paged_attn_decode_fp8: as paged_attn_decode, with desc->dtype the type of q and out
+ * (PKV_F16 or PKV_BF16); the same workspace rule (pkv_attn_workspace_bytes(desc)).
+ * Scores and the weighted sum run on the codes widened to f16 with fp32 accumulation; the
+ * K scale multiplies the scores and the V scale the output.
+ */
+pkv_status kv_write_fp8(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
+                        const int64_t *slot_mapping, int32_t num_tokens, const float *k_scale,
+                        const float *v_scale, void *k_pool, void *v_pool, void *stream);
+pkv_status paged_attn_decode_fp8(const pkv_attn_desc *desc, const void *q, const void *k_pool,
+                                 const void *v_pool, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables,
+                                 const int32_t *context_lens, float scale, void *out,
+                                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Allocation-free variant of paged_attn_decode.  The paper has no counterpart: this entry

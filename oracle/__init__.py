@@ -55,6 +55,15 @@ def lib():
         L.orc_kv_copy_blocks.restype = i32
         L.orc_kv_swap.argtypes = [i32, vp, vp, vp, i32, vp, vp, i32, ctypes.c_size_t]
         L.orc_kv_swap.restype = i32
+        L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_to_f64.restype = f64
+        L.orc_f32_to_e4m3.argtypes = [ctypes.c_float]
+        L.orc_f32_to_e4m3.restype = ctypes.c_uint8
+        L.orc_kv_write_fp8.argtypes = [i32] * 5 + [vp, vp, i32, vp, vp, vp, vp, vp]
+        L.orc_kv_write_fp8.restype = i32
+        L.orc_paged_attn_decode_fp8.argtypes = [i32] * 7 + [vp, i32, vp, vp, vp, vp, vp, vp,
+                                                            f64, vp, i32, vp, i32]
+        L.orc_paged_attn_decode_fp8.restype = i32
         _lib = L
     return _lib
 
@@ -197,3 +206,61 @@ def kv_swap(pairs, src_k, src_v, dst_k, dst_v):
     rc = lib().orc_kv_swap(pr.shape[0], _ptr(pr), _ptr(src_k), _ptr(src_v), src_k.shape[0],
                            _ptr(dst_k), _ptr(dst_v), dst_k.shape[0], bb)
     _check(rc, "kv_swap")
+
+
+# ---- FP8 (E4M3) KV cache: per-head fp32 scales, K [NB,Hkv,B,D], V [NB,Hkv,D,B] codes ------
+def e4m3_to_f64(code: int) -> float:
+    return lib().orc_e4m3_to_f64(int(code) & 0xFF)
+
+
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().orc_f32_to_e4m3(float(x)))
+
+
+def kv_write_fp8(k_new, v_new, slot_mapping, k_scale, v_scale, k_pool, v_pool, dtype):
+    """Quantise new K/V rows [T, Hkv, D] of ``dtype`` into uint8 E4M3 pools, in place:
+    K pool [NB, Hkv, B, D], V pool [NB, Hkv, D, B] (transposed within the block; slot p of
+    a row holds token 2*(p//4) + p%2 + 8*((p//2)%2))."""
+    k_new = _as_bits(k_new, dtype)
+    v_new = _as_bits(v_new, dtype)
+    T, Hkv, D = k_new.shape
+    NB, Hkv2, B, D2 = k_pool.shape
+    if (Hkv2, D2) != (Hkv, D) or v_pool.shape != (NB, Hkv, D, B):
+        raise ValueError("shape mismatch")
+    for a in (k_pool, v_pool):
+        if a.dtype != np.uint8 or not a.flags.c_contiguous:
+            raise TypeError("pools must be C-contiguous uint8")
+    ks = np.ascontiguousarray(k_scale, np.float32)
+    vs = np.ascontiguousarray(v_scale, np.float32)
+    sm = np.ascontiguousarray(slot_mapping, np.int64)
+    rc = lib().orc_kv_write_fp8(T, Hkv, D, B, NB, _ptr(k_new), _ptr(v_new), DTYPES[dtype],
+                                _ptr(sm), _ptr(ks), _ptr(vs), _ptr(k_pool), _ptr(v_pool))
+    _check(rc, "kv_write_fp8")
+
+
+def paged_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, block_tables, context_lens,
+                          scale, q_dtype, rows=None, nthreads=None):
+    """Decode attention over E4M3 pools (values code * per-head scale), exact in fp64."""
+    q = _as_bits(q, q_dtype)
+    S, Hq, D = q.shape
+    NB, Hkv, B, D2 = k_pool.shape
+    if D2 != D or v_pool.shape != (NB, Hkv, D, B):
+        raise ValueError("shape mismatch")
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    ks = np.ascontiguousarray(k_scale, np.float32)
+    vs = np.ascontiguousarray(v_scale, np.float32)
+    if rows is None:
+        out = np.empty((S, Hq, D), np.float64)
+        rr, n = None, 0
+    else:
+        rr = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 2)
+        n = rr.shape[0]
+        out = np.empty((n, D), np.float64)
+    rc = lib().orc_paged_attn_decode_fp8(S, Hq, Hkv, D, B, NB, bt.shape[1], _ptr(q),
+                                         DTYPES[q_dtype], _ptr(np.ascontiguousarray(k_pool)),
+                                         _ptr(np.ascontiguousarray(v_pool)), _ptr(ks), _ptr(vs),
+                                         _ptr(bt), _ptr(lens), float(scale), _ptr(rr), n,
+                                         _ptr(out), nthreads or num_threads())
+    _check(rc, "paged_attn_decode_fp8")
+    return out

@@ -341,3 +341,148 @@ int orc_kv_swap(int P, const int32_t *pairs, const void *src_k, const void *src_
     }
     return err;
 }
+
+/* ---------------------------------------------------------------------------------------
+ * FP8 (E4M3) KV cache.  "Memory Optimization in LLM Serving with PagedAttention", section
+ * "Broader Context: vLLM, TGI, and TensorRT-LLM": paged KV caches are also kept in INT8/FP8
+ * to cut memory.  The scheme (our reading; the page names no format): each KV head has one
+ * fp32 scale for K and one for V; a value x is stored as the E4M3 code of x / scale (fp32
+ * division, round to nearest even, saturating to +-448); its value is code * scale.
+ * K blocks keep the [block][head][token][dim] layout; V blocks are stored transposed within
+ * the block, [block][head][dim][slot], slot p holding token 2*(p/4) + p%2 + 8*((p/2)%2).
+ * ------------------------------------------------------------------------------------- */
+
+/* E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits; no infinities; S.1111.111 is
+ * NaN; largest finite 448. */
+double orc_e4m3_to_f64(uint8_t c) {
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xf;
+    int f = c & 0x7;
+    double v;
+    if (e == 15 && f == 7) return NAN;
+    if (e == 0) v = ldexp((double)f, -9);              /* f * 2^(1-7-3) */
+    else v = ldexp((double)(8 + f), e - 10);           /* (1 + f/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code of a float (ties to even), saturating to +-448; NaN gives 0x7F. */
+uint8_t orc_f32_to_e4m3(float x) {
+    if (x != x) return 0x7f;
+    uint8_t sign = (x < 0 || (x == 0 && signbit(x))) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7e;
+    int code;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal grid, step 2^-9; the carry out of 7 is the smallest normal code 8 */
+        code = (int)nearbyint(a / ldexp(1.0, -9));
+    } else {
+        int ex;
+        frexp(a, &ex);                                /* a = m * 2^ex, m in [0.5, 1) */
+        int e = ex - 1;                               /* a in [2^e, 2^(e+1)) */
+        int n = (int)nearbyint(a / ldexp(1.0, e - 3)); /* in [8, 16] */
+        code = ((e + 7) << 3) + (n - 8);              /* n = 16 carries into e + 1 */
+    }
+    if (code > 0x7e) code = 0x7e;
+    return sign | (uint8_t)code;
+}
+
+/* Transposed V rows hold the block's 16 tokens in a fixed slot order: slot p holds token
+ * 2*(p/4) + p%2 + 8*((p/2)%2).  The slot of token t is found by trying every slot. */
+static int orc_v_slot(int t) {
+    for (int p = 0; p < 16; ++p)
+        if (2 * (p / 4) + p % 2 + 8 * ((p / 2) % 2) == t) return p;
+    return -1;
+}
+
+/* Value of new element i of dtype (f16 / bf16 / f32) as a float (exact). */
+static float orc_load_f32(const void *base, int dtype, size_t i) {
+    return (float)orc_load(base, dtype, i);
+}
+
+/*
+ * kv_write into FP8 pools: for token t and head h with slot s (s = -1 skips),
+ *   k_pool[s/B][h][s%B][d] = e4m3(k_new[t][h][d] / k_scale[h])
+ *   v_pool[s/B][h][d][s%B] = e4m3(v_new[t][h][d] / v_scale[h])
+ */
+int orc_kv_write_fp8(int T, int Hkv, int D, int B, int NB, const void *k_new,
+                     const void *v_new, int new_dtype, const int64_t *slot_mapping,
+                     const float *k_scale, const float *v_scale, uint8_t *k_pool,
+                     uint8_t *v_pool) {
+    if (T < 0 || Hkv < 1 || D < 1 || B != 16 || NB < 0 || !orc_elem_size(new_dtype))
+        return ORC_BAD_ARG;
+    int err = ORC_OK;
+    for (int t = 0; t < T; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot == -1) continue;
+        if (slot < 0 || slot >= (int64_t)NB * B) { err = ORC_BAD_SLOT; continue; }
+        int64_t blk = slot / B;
+        int off = (int)(slot % B);
+        for (int h = 0; h < Hkv; ++h)
+            for (int d = 0; d < D; ++d) {
+                size_t src = ((size_t)t * Hkv + h) * D + d;
+                float kq = orc_load_f32(k_new, new_dtype, src) / k_scale[h];
+                float vq = orc_load_f32(v_new, new_dtype, src) / v_scale[h];
+                k_pool[(((size_t)blk * Hkv + h) * B + off) * D + d] = orc_f32_to_e4m3(kq);
+                v_pool[(((size_t)blk * Hkv + h) * D + d) * B + orc_v_slot(off)] =
+                    orc_f32_to_e4m3(vq);
+            }
+    }
+    return err;
+}
+
+/* Decode attention over FP8 pools (layouts above), exact two-pass softmax in fp64 on the
+ * dequantised values code * scale.  Same row contract as orc_paged_attn_decode. */
+int orc_paged_attn_decode_fp8(int S, int Hq, int Hkv, int D, int B, int NB, int maxB,
+                              const void *q, int q_dtype, const uint8_t *k_pool,
+                              const uint8_t *v_pool, const float *k_scale,
+                              const float *v_scale, const int32_t *block_tables,
+                              const int32_t *context_lens, double scale, const int32_t *rows,
+                              int nrows, double *out, int nthreads) {
+    if (S < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || B != 16 || NB < 0 || maxB < 0 ||
+        !orc_elem_size(q_dtype))
+        return ORC_BAD_ARG;
+    int n = rows ? nrows : S * Hq;
+    int err = ORC_OK;
+    if (nthreads < 1) nthreads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+    for (int r = 0; r < n; ++r) {
+        int s = rows ? rows[2 * r] : r / Hq;
+        int h = rows ? rows[2 * r + 1] : r % Hq;
+        double *o = out + (size_t)r * D;
+        int rc = (s < 0 || s >= S || h < 0 || h >= Hq) ? ORC_BAD_ARG
+                 : orc_check_seq(s, B, NB, maxB, block_tables, context_lens);
+        if (rc) {
+            for (int d = 0; d < D; ++d) o[d] = NAN;
+#pragma omp critical
+            { if (!err) err = rc; }
+            continue;
+        }
+        int L = context_lens[s], hk = h / (Hq / Hkv);
+        double ks = k_scale[hk], vs = v_scale[hk];
+        double *x = (double *)malloc(sizeof(double) * (size_t)L);
+        double M = -INFINITY;
+        for (int t = 0; t < L; ++t) {
+            int64_t p = block_tables[(size_t)s * maxB + t / B];
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d)
+                acc += orc_load(q, q_dtype, ((size_t)s * Hq + h) * D + d) *
+                       (orc_e4m3_to_f64(k_pool[(((size_t)p * Hkv + hk) * B + t % B) * D + d]) * ks);
+            x[t] = scale * acc;
+            if (x[t] > M) M = x[t];
+        }
+        double den = 0.0;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        for (int t = 0; t < L; ++t) {
+            int64_t p = block_tables[(size_t)s * maxB + t / B];
+            double w = exp(x[t] - M);
+            den += w;
+            for (int d = 0; d < D; ++d)
+                o[d] += w * (orc_e4m3_to_f64(
+                                 v_pool[(((size_t)p * Hkv + hk) * D + d) * B + orc_v_slot(t % B)]) *
+                             vs);
+        }
+        for (int d = 0; d < D; ++d) o[d] /= den;
+        free(x);
+    }
+    return err;
+}

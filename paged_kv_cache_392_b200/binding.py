@@ -18,7 +18,8 @@ STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID", 2: "PKV_ERR_OOM", 3: "PKV_ERR_UNSUP
           4: "PKV_ERR_CUDA", 5: "PKV_ERR_NOT_FOUND"}
 FAULT_BITS = {0x1: "bad context length", 0x2: "bad block id", 0x4: "bad slot",
               0x8: "bad copy pair", 0x10: "barrier wait timed out"}
-DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2}
+DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.uint8: 3}
+PKV_FP8_E4M3 = 3
 BLOCK_SIZE = 16
 
 # Every symbol include/pkv.h declares.
@@ -29,7 +30,7 @@ EXPORTS = [
     "pkv_bm_free_seq", "pkv_bm_block_table", "pkv_bm_block_tables", "pkv_bm_seq_len",
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
-    "pkv_bm_is_swapped", "pkv_bm_num_host_free",
+    "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
 ]
 
 
@@ -94,6 +95,9 @@ def lib():
         "pkv_bm_swap_in": ([vp, i64, vp, i32, P(i32)], i32),
         "pkv_bm_is_swapped": ([vp, i64, P(i32)], i32),
         "pkv_bm_num_host_free": ([vp], i32),
+        "kv_write_fp8": ([dp, vp, vp, vp, i32, vp, vp, vp, vp, vp], i32),
+        "paged_attn_decode_fp8": ([dp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz,
+                                   vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -282,6 +286,60 @@ def kv_swap_in(pairs, host_k, host_v, k_pool, v_pool, stream=None):
     _check(lib().kv_swap_in(ctypes.byref(desc), _ptr(pairs), pairs.shape[0], _ptr(host_k),
                             _ptr(host_v), host_k.shape[0], _ptr(k_pool), _ptr(v_pool),
                             _stream(stream, k_pool.device)))
+
+
+def _fp8_pools(k_pool, v_pool):
+    """FP8 pools: K [NB, H_kv, 16, D] and V [NB, H_kv, D, 16], uint8 E4M3 codes."""
+    _dev(k_pool, "k_pool", torch.uint8)
+    _dev(v_pool, "v_pool", torch.uint8)
+    if k_pool.dim() != 4 or v_pool.shape != (k_pool.shape[0], k_pool.shape[1],
+                                             k_pool.shape[3], k_pool.shape[2]):
+        raise ValueError("FP8 pools: K [NB, H_kv, 16, D], V [NB, H_kv, D, 16]")
+    return k_pool.shape
+
+
+def kv_write_fp8(k_new, v_new, slot_mapping, k_scale, v_scale, k_pool, v_pool, stream=None):
+    """Quantise new K/V rows [T, H_kv, D] (f16/bf16/f32) into the FP8 pools' slots."""
+    NB, Hkv, Bs, D = _fp8_pools(k_pool, v_pool)
+    _dev(k_new, "k_new")
+    _dev(v_new, "v_new", k_new.dtype)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    _dev(k_scale, "k_scale", torch.float32)
+    _dev(v_scale, "v_scale", torch.float32)
+    T = k_new.shape[0]
+    if k_new.shape != (T, Hkv, D) or v_new.shape != k_new.shape or \
+            slot_mapping.shape != (T,) or k_scale.shape != (Hkv,) or v_scale.shape != (Hkv,):
+        raise ValueError("k_new/v_new [T, H_kv, D], slot_mapping [T], scales [H_kv] expected")
+    desc = make_desc(0, Hkv, Hkv, D, NB, 1, k_new.dtype, 0, Bs)
+    _check(lib().kv_write_fp8(ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+                              T, _ptr(k_scale), _ptr(v_scale), _ptr(k_pool), _ptr(v_pool),
+                              _stream(stream, k_pool.device)))
+
+
+def paged_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, block_tables, context_lens,
+                          scale, out=None, workspace=None, partition_tokens=0, stream=None):
+    """Decode attention over FP8 pools; q/out f16 or bf16 [S, H_q, D]."""
+    NB, Hkv, Bs, D = _fp8_pools(k_pool, v_pool)
+    _dev(q, "q")
+    _dev(k_scale, "k_scale", torch.float32)
+    _dev(v_scale, "v_scale", torch.float32)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    S, Hq, Dq = q.shape
+    if Dq != D or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("q [S,Hq,D], block_tables [S,maxB], context_lens [S] expected")
+    desc = make_desc(S, Hq, Hkv, D, NB, block_tables.shape[1], q.dtype, partition_tokens, Bs)
+    if out is None:
+        out = torch.empty_like(q)
+    need = attn_workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().paged_attn_decode_fp8(ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool),
+                                       _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                                       _ptr(context_lens), float(scale), _ptr(out),
+                                       _ptr(workspace), nbytes, _stream(stream, q.device)))
+    return out
 
 
 def device_faults(clear=True, stream=None, device=None):

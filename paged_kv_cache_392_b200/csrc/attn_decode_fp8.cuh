@@ -1,0 +1,442 @@
+// FP8 (E4M3) paged KV cache: quantising write and tensor-core decode (sm_100a).
+//
+// "Memory Optimization in LLM Serving with PagedAttention", section "Broader Context: vLLM,
+// TGI, and TensorRT-LLM": paged KV caches are also kept in INT8/FP8 to cut memory.  The page
+// fixes no format; this library's reading:
+//   * each KV head has one fp32 scale for K and one for V; element x is stored as the E4M3
+//     code of x / scale (fp32 division, round to nearest even, saturating to +-448) and
+//     means code * scale;
+//   * K blocks: [block][kv head][16 tokens][D] bytes (as the 16-bit pools);
+//   * V blocks: [block][kv head][D][16 slots] bytes -- transposed, and slot p of a row holds
+//     token v_slot_token(p) (below), so that a 16-byte row read by one ldmatrix lane quarter
+//     gives the token pairs the P.V tile wants.
+// Decode: q.K^T runs on m16n8k32 E4M3 tensor-core tiles straight from the K codes, with each
+// query row prescaled by a power of two and split into two E4M3 terms (hi + residual, about
+// bfloat16 precision); P.V widens the V codes exactly to f16 (every E4M3 value is an f16
+// value) for m16n8k16 f16 tiles.  Accumulation is fp32; the K scale (and the q prescale) is
+// folded into the softmax scale and the V scale into the output.  Only D = 128 is built.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp8.h>
+
+#include <type_traits>
+
+#include "attn_decode_tc.cuh"
+
+namespace pkv {
+
+// Slot p of a transposed V row holds token t = 2*(p>>2) + (p&1) + 8*((p>>1)&1); its inverse:
+__host__ __device__ __forceinline__ int v_slot_of_token(int t) {
+    return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
+}
+
+// Two E4M3 codes (low byte first) to an f16x2 register, exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// D = A * B + C for one m16n8k32 tile of E4M3 codes, fp32 accumulators.
+__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two floats to an f16x2 register (round to nearest even).
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+    return pack2<false>(lo, hi);
+}
+
+struct DecodeFp8Params {
+    DecodeParams base;        // q/out/workspace/shape (k_pool/v_pool: the E4M3 pools)
+    const float *k_scale;     // [H_kv]
+    const float *v_scale;     // [H_kv]
+};
+
+template <int W, int NSW>
+struct DecodeFp8Cfg {
+    static constexpr int D = 128;
+    static constexpr int CHUNK = kBlock * D;      // bytes of one (block, head) of K or of V
+    static constexpr int STAGE = 2 * CHUNK;       // K (swizzled box) then V (transposed)
+    static constexpr int RING = W * NSW * STAGE;
+    static constexpr int BARS = W * NSW * 8;
+    static constexpr int KSTEPS = D / 16;
+    template <int G>
+    static constexpr int smem() { return 1024 + RING + BARS + W * G * (D + 2) * 4; }
+};
+
+// T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.
+template <typename T, int G, int W, int NSW>
+__global__ void __launch_bounds__(W * 32)
+paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
+                             const DecodeFp8Params fp) {
+    using C = DecodeFp8Cfg<W, NSW>;
+    constexpr int D = C::D, CHUNK = C::CHUNK, KSTEPS = C::KSTEPS;
+    constexpr unsigned FULL = 0xffffffffu;
+    const DecodeParams &p = fp.base;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    pdl_launch_dependents();
+
+    const int bid = blockIdx.x;
+    const int part = bid % p.pmax;
+    const int rest = bid / p.pmax;
+    const int hk = rest % p.Hkv;
+    const int s = rest / p.Hkv;
+
+    const int L = p.context_lens[s];
+    if (L < 1 || L > p.maxB * kBlock) {
+        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, 0x1u);
+        return;
+    }
+    const int nblk = (L + kBlock - 1) / kBlock;
+    const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
+    if (part >= nparts) return;
+    const int j0 = part * p.part_blocks;
+    const int nb = min(nblk, j0 + p.part_blocks) - j0;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2;
+    const int tq = lane & 3;
+    const int nbw = nb > warp ? (nb - warp + W - 1) / W : 0;
+
+    unsigned char *ring = smem + warp * NSW * C::STAGE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::RING) + warp * NSW;
+    float *mo = reinterpret_cast<float *>(smem + C::RING + C::BARS);
+    float *mml = mo + W * G * D;
+
+    if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < NSW; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        if (warp == 0) prefetch_tmap(&tmk);
+    }
+    __syncwarp();
+
+    const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const char *vbase = static_cast<const char *>(p.v_pool);
+    const uint64_t policy = l2_evict_first_policy();
+    int tab_chunk = 0;
+    int32_t tab = lane < nbw ? btrow[(size_t)W * lane] : 0;
+
+    auto issue = [&](int i) {
+        if ((i >> 5) != tab_chunk) {
+            tab_chunk = i >> 5;
+            const int li = (tab_chunk << 5) + lane;
+            tab = li < nbw ? btrow[(size_t)W * li] : 0;
+        }
+        const int32_t phys = __shfl_sync(FULL, tab, i & 31);
+        if (lane == 0) {
+            uint64_t *bar = &bars[i % NSW];
+            unsigned char *dst = ring + (i % NSW) * C::STAGE;
+            if ((unsigned)phys < (unsigned)p.NB) {
+                const int32_t row = (phys * p.Hkv + hk) * kBlock;
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(bar, 2 * CHUNK);
+                tma_load_2d(dst, &tmk, 0, row, bar, policy);
+                bulk_g2s(dst + CHUNK, vbase + (size_t)(phys * p.Hkv + hk) * CHUNK, CHUNK, bar,
+                         policy);
+            } else {
+                atomicOr(&g_faults, 0x2u);
+                mbar_arrive(bar);
+            }
+        }
+    };
+
+    const int npro = nbw < NSW ? nbw : NSW;
+    for (int i = 0; i < npro; ++i) issue(i);
+    int issued = npro;
+
+    // Q^T as the B operand of S^T = K Q^T on E4M3 tiles (m16n8k32): each query row is scaled
+    // by a power of two qf (its largest |q| lands in [128, 256)) and split into two E4M3
+    // terms, hi = e4m3(q*qf) and lo = e4m3(q*qf - hi), which carry about 8 significant bits
+    // (a bfloat16 q exactly, up to subnormal tails).  Lane (g, tq) holds head g, dims
+    // 32j+4tq..+3 (b0) and 32j+16+4tq..+3 (b1) of k-step j.
+    constexpr int K32 = D / 32;
+    uint32_t qhi[K32][2], qlo[K32][2];
+    float qf_mine = 1.f;
+    {
+        const bool hv = g < G;
+        const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
+        float qv[K32][2][4];
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < K32; ++j)
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v = 0.f;
+                    if (hv) {
+                        if constexpr (std::is_same<T, __half>::value)
+                            v = __half2float(qrow[32 * j + 16 * b + 4 * tq + e]);
+                        else
+                            v = __bfloat162float(qrow[32 * j + 16 * b + 4 * tq + e]);
+                    }
+                    qv[j][b][e] = v;
+                    amax = fmaxf(amax, fabsf(v));
+                }
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+        if (amax > 0.f && amax < INFINITY) {
+            int ex;
+            frexpf(amax, &ex);                  // amax < 2^ex
+            qf_mine = ldexpf(1.f, 8 - ex);      // amax * qf in [128, 256)
+        }
+#pragma unroll
+        for (int j = 0; j < K32; ++j)
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                uint32_t hi = 0u, lo = 0u;
+#pragma unroll
+                for (int e = 0; e < 4; e += 2) {
+                    const float2 x = make_float2(qv[j][b][e] * qf_mine, qv[j][b][e + 1] * qf_mine);
+                    const __nv_fp8x2_storage_t h2 = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h2, __NV_E4M3);
+                    const float2 r = make_float2(x.x - __half2float(__half(hr.x)),
+                                                 x.y - __half2float(__half(hr.y)));
+                    const __nv_fp8x2_storage_t l2 = __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
+                    hi |= static_cast<uint32_t>(h2) << (8 * e);
+                    lo |= static_cast<uint32_t>(l2) << (8 * e);
+                }
+                qhi[j][b] = hi;
+                qlo[j][b] = lo;
+            }
+    }
+
+    float o[KSTEPS][4];
+#pragma unroll
+    for (int i = 0; i < KSTEPS; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    // score scales of this lane's heads 2tq, 2tq+1: softmax scale * K scale / q prescale
+    const float slk = p.scale_log2 * fp.k_scale[hk];
+    const float sl0 = slk / __shfl_sync(FULL, qf_mine, (2 * tq) * 4);
+    const float sl1 = slk / __shfl_sync(FULL, qf_mine, (2 * tq + 1) * 4);
+
+    // ldmatrix roles.  K rows (tokens) in natural order; matrix mi of a k-step pair covers
+    // tokens 8*(mi&1).. and 16-byte chunk 2j+(mi>>1).  V^T rows are head dims, two m-tiles
+    // (32 rows) per x4.
+    const int k_tok = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int k_c = lane >> 4;
+    const int v_row = lane;  // row within the 32-row group
+
+    bool dead = false;
+    int i = 0;
+    for (; i < nbw; ++i) {
+        const int st = i % NSW;
+        if (!mbar_wait_bounded(&bars[st], (uint32_t)(i / NSW) & 1u, kWaitTimeoutNs)) {
+            if (lane == 0) atomicOr(&g_faults, 0x10u);
+            dead = true;
+            break;
+        }
+        unsigned char *Ks = ring + st * C::STAGE;
+        unsigned char *Vs = Ks + CHUNK;
+        const int jb = j0 + warp + W * i;
+        const int nvalid = min(kBlock, L - jb * kBlock);
+        if (nvalid < kBlock) {
+            // zero the V^T slots of tokens past the context (their codes may be NaN)
+            uint32_t keep[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int t = 0; t < kBlock; ++t)
+                if (t < nvalid) {
+                    const int sp = v_slot_of_token(t);
+                    keep[sp >> 2] |= 0xffu << (8 * (sp & 3));
+                }
+            for (int r = lane; r < D; r += 32) {
+                uint4 *row = reinterpret_cast<uint4 *>(Vs + r * 16);
+                uint4 v = *row;
+                v.x &= keep[0];
+                v.y &= keep[1];
+                v.z &= keep[2];
+                v.w &= keep[3];
+                *row = v;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+
+        // ---- S^T = K Q^T on E4M3 tiles: K codes go from ldmatrix straight into the A
+        // fragments (row g / g+8, k 4tq..4tq+3 and 16+4tq..16+4tq+3 of each 32-dim step)
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t kb = smem_u32(Ks);
+#pragma unroll
+        for (int j = 0; j < K32; ++j) {
+            const int c = 2 * j + k_c;  // 16-byte chunk of the 128-byte row
+            uint32_t a[4];
+            ldmatrix_x4(a, kb + k_tok * 128 + ((c ^ (k_tok & 7)) << 4));
+            mma_16832_e4m3(sacc, a, qhi[j][0], qhi[j][1]);
+            mma_16832_e4m3(sacc, a, qlo[j][0], qlo[j][1]);
+        }
+
+        // ---- online softmax (lane: tokens g, g+8 of heads 2tq, 2tq+1) --------------------
+        const float x0 = g < nvalid ? sacc[0] * sl0 : -INFINITY;
+        const float x1 = g < nvalid ? sacc[1] * sl1 : -INFINITY;
+        const float x2 = g + 8 < nvalid ? sacc[2] * sl0 : -INFINITY;
+        const float x3 = g + 8 < nvalid ? sacc[3] * sl1 : -INFINITY;
+        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
+            bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
+        }
+        const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
+        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
+        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
+        const float a0 = exp2f(m_run[0] - mn0), a1 = exp2f(m_run[1] - mn1);
+        float s0 = p0 + p2, s1 = p1 + p3;
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            s0 += __shfl_xor_sync(FULL, s0, m);
+            s1 += __shfl_xor_sync(FULL, s1, m);
+        }
+        l_run[0] = l_run[0] * a0 + s0;
+        l_run[1] = l_run[1] * a1 + s1;
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+
+        // P^T fragments: b0 holds tokens 2tq, 2tq+1 and b1 tokens 8+2tq, 9+2tq of head g,
+        // which are the slots 4tq..4tq+3 a lane reads from a V^T row.
+        const uint32_t b0 = movmatrix_trans(f32x2_to_f16x2(p0, p1));
+        const uint32_t b1 = movmatrix_trans(f32x2_to_f16x2(p2, p3));
+
+        if (__any_sync(FULL, a0 != 1.f || a1 != 1.f)) {
+#pragma unroll
+            for (int t = 0; t < KSTEPS; ++t) {
+                o[t][0] *= a0;
+                o[t][1] *= a1;
+                o[t][2] *= a0;
+                o[t][3] *= a1;
+            }
+        }
+
+        // ---- O^T += V^T P^T -----------------------------------------------------------------
+        const uint32_t vb = smem_u32(Vs);
+#pragma unroll
+        for (int t2 = 0; t2 < KSTEPS / 2; ++t2) {
+            uint32_t r[4];
+            ldmatrix_x4(r, vb + (32 * t2 + v_row) * 16);
+            // r[0]: dims 32t2+0..7, r[1]: +8..15 (m-tile 2t2); r[2], r[3]: m-tile 2t2+1
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t a[4];
+                a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] & 0xffffu));
+                a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] >> 16));
+                a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] & 0xffffu));
+                a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] >> 16));
+                mma_16816<false>(o[2 * t2 + h], a, b0, b1);
+            }
+        }
+        __syncwarp();
+
+        if (issued < nbw) {
+            issue(issued);
+            ++issued;
+        }
+    }
+    if (dead) {
+        for (int b = i; b < issued; ++b)
+            (void)mbar_wait_bounded(&bars[b % NSW], (uint32_t)(b / NSW) & 1u, kWaitTimeoutNs);
+        m_run[0] = m_run[1] = -INFINITY;
+        l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+        for (int t = 0; t < KSTEPS; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+    }
+
+    const float vsc = fp.v_scale[hk];
+    const int h0 = 2 * tq, h1 = 2 * tq + 1;
+    if (h0 < G) {
+        float *dst = mo + (warp * G + h0) * D;
+#pragma unroll
+        for (int t = 0; t < KSTEPS; ++t) {
+            dst[16 * t + g] = o[t][0] * vsc;
+            dst[16 * t + g + 8] = o[t][2] * vsc;
+        }
+        if (g == 0) {
+            mml[(warp * G + h0) * 2] = m_run[0];
+            mml[(warp * G + h0) * 2 + 1] = l_run[0];
+        }
+    }
+    if (h1 < G) {
+        float *dst = mo + (warp * G + h1) * D;
+#pragma unroll
+        for (int t = 0; t < KSTEPS; ++t) {
+            dst[16 * t + g] = o[t][1] * vsc;
+            dst[16 * t + g + 8] = o[t][3] * vsc;
+        }
+        if (g == 0) {
+            mml[(warp * G + h1) * 2] = m_run[1];
+            mml[(warp * G + h1) * 2 + 1] = l_run[1];
+        }
+    }
+    __syncthreads();
+    merge_and_store<T, D, G, W>(p, mo, mml, s, hk, part, nparts);
+}
+
+// ---- quantising write ----------------------------------------------------------------------
+struct KvWriteFp8Params {
+    const void *k_new;  // [T][H_kv][D] of the new-value type
+    const void *v_new;
+    const int64_t *slot_mapping;
+    const float *k_scale;
+    const float *v_scale;
+    uint8_t *k_pool;    // [NB][H_kv][16][D]
+    uint8_t *v_pool;    // [NB][H_kv][D][16] (slot order v_slot_of_token)
+    int32_t T, Hkv, NB, D;
+};
+
+template <typename T>
+__device__ __forceinline__ float load_elem(const void *base, int64_t i) {
+    if constexpr (std::is_same<T, float>::value)
+        return static_cast<const float *>(base)[i];
+    else if constexpr (std::is_same<T, __half>::value)
+        return __half2float(static_cast<const __half *>(base)[i]);
+    else
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(base)[i]);
+}
+
+// One thread per (token, head, pair of dims): codes of x / scale, RNE, saturating.
+template <typename T>
+__global__ void __launch_bounds__(256) kv_write_fp8_kernel(const KvWriteFp8Params p) {
+    const int64_t pairs = (int64_t)p.T * p.Hkv * (p.D / 2);
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= pairs) return;
+    const int d = 2 * (int)(idx % (p.D / 2));
+    const int64_t th = idx / (p.D / 2);
+    const int h = (int)(th % p.Hkv);
+    const int64_t t = th / p.Hkv;
+    const int64_t slot = p.slot_mapping[t];
+    if (slot == -1) return;
+    if (slot < 0 || slot >= (int64_t)p.NB * 16) {
+        if (h == 0 && d == 0) atomicOr(&g_faults, 0x4u);
+        return;
+    }
+    const int64_t blk = slot >> 4;
+    const int off = (int)(slot & 15);
+    const int64_t src = th * p.D + d;
+    const float ks = p.k_scale[h], vs = p.v_scale[h];
+    const float2 kx = make_float2(load_elem<T>(p.k_new, src) / ks,
+                                  load_elem<T>(p.k_new, src + 1) / ks);
+    const float2 vx = make_float2(load_elem<T>(p.v_new, src) / vs,
+                                  load_elem<T>(p.v_new, src + 1) / vs);
+    const __nv_fp8x2_storage_t kc = __nv_cvt_float2_to_fp8x2(kx, __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t vc = __nv_cvt_float2_to_fp8x2(vx, __NV_SATFINITE, __NV_E4M3);
+    const int64_t hb = blk * p.Hkv + h;
+    *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + (hb * 16 + off) * p.D + d) = kc;
+    const int sp = v_slot_of_token(off);
+    p.v_pool[(hb * p.D + d) * 16 + sp] = static_cast<uint8_t>(vc & 0xffu);
+    p.v_pool[(hb * p.D + d + 1) * 16 + sp] = static_cast<uint8_t>(vc >> 8);
+}
+
+}  // namespace pkv

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "attn_decode.cuh"
+#include "attn_decode_fp8.cuh"
 #include "attn_decode_tc.cuh"
 #include "kv_ops.cuh"
 #include "pkv_internal.h"
@@ -24,7 +25,10 @@ constexpr int kMaxDevices = 64;
 constexpr int kDefaultPartitionTokens = pkv::kDefaultPartitionTokens;
 
 int elem_size(int32_t dtype) {
-    return dtype == PKV_F32 ? 4 : (dtype == PKV_F16 || dtype == PKV_BF16) ? 2 : 0;
+    return dtype == PKV_F32 ? 4
+           : (dtype == PKV_F16 || dtype == PKV_BF16) ? 2
+           : dtype == PKV_FP8_E4M3 ? 1
+           : 0;
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -55,6 +59,8 @@ struct Split {
 pkv_status check_attn_desc(const pkv_attn_desc *d, const char *fn, Split *sp) {
     pkv_status st = check_pool_desc(d, fn);
     if (st) return st;
+    if (d->dtype == PKV_FP8_E4M3)
+        return fail(PKV_ERR_INVALID, "%s: desc->dtype is the q/out type (f32, f16, bf16)", fn);
     if (d->num_seqs < 0) return fail(PKV_ERR_INVALID, "%s: num_seqs < 0", fn);
     if (d->num_q_heads < 1 || d->num_q_heads % d->num_kv_heads)
         return fail(PKV_ERR_INVALID, "%s: num_q_heads %d not a multiple of num_kv_heads %d", fn,
@@ -316,6 +322,8 @@ pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_
     const char *fn = "kv_write";
     pkv_status st = check_pool_desc(desc, fn);
     if (st) return st;
+    if (desc->dtype == PKV_FP8_E4M3)
+        return fail(PKV_ERR_INVALID, "%s: FP8 pools are written by kv_write_fp8", fn);
     if (num_tokens < 0) return fail(PKV_ERR_INVALID, "%s: num_tokens < 0", fn);
     if (num_tokens == 0) return PKV_OK;
     if (!k_new || !v_new || !slot_mapping || !k_pool || !v_pool)
@@ -365,6 +373,168 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
     dim3 grid((unsigned)(2 * num_pairs), (unsigned)slices);
     pkv::kv_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
     return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+}  // extern "C"
+
+// ---- FP8 (E4M3) KV cache --------------------------------------------------------------------
+namespace {
+
+constexpr int kFp8Warps = PKV_DECODE_TC_WARPS;
+constexpr int kFp8Stages = PKV_DECODE_TC_STAGES;
+
+pkv_status fp8_k_tensor_map(CUtensorMap *m, const void *pool, int64_t rows, const char *fn) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(PKV_ERR_CUDA, "%s: cuTensorMapEncodeTiled unavailable", fn);
+    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128};
+    const cuuint32_t box[2] = {128, (cuuint32_t)pkv::kBlock};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(pool), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PKV_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed (%d)", fn, (int)r);
+    return PKV_OK;
+}
+
+template <typename T, int G>
+pkv_status launch_decode_fp8(const pkv::DecodeFp8Params &fp, cudaStream_t stream) {
+    using Cfg = pkv::DecodeFp8Cfg<kFp8Warps, kFp8Stages>;
+    constexpr int kSmem = Cfg::template smem<G>();
+    auto kern = pkv::paged_attn_decode_fp8_kernel<T, G, kFp8Warps, kFp8Stages>;
+    static std::atomic<bool> done[kMaxDevices];
+    pkv_status st = ensure_smem(kern, kSmem, done, "paged_attn_decode_fp8");
+    if (st) return st;
+    CUtensorMap tmk;
+    st = fp8_k_tensor_map(&tmk, fp.base.k_pool, (int64_t)fp.base.NB * fp.base.Hkv * pkv::kBlock,
+                          "paged_attn_decode_fp8");
+    if (st) return st;
+    const unsigned grid = (unsigned)((int64_t)fp.base.S * fp.base.Hkv * fp.base.pmax);
+    kern<<<grid, kFp8Warps * 32, kSmem, stream>>>(tmk, fp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode_fp8", "decode launch");
+    return launch_reduce_if_split(fp.base, stream, pkv::lse_reduce_kernel<T, 128>);
+}
+
+template <typename T>
+pkv_status dispatch_fp8(int g, const pkv::DecodeFp8Params &fp, cudaStream_t stream) {
+    switch (g) {
+    case 1: return launch_decode_fp8<T, 1>(fp, stream);
+    case 2: return launch_decode_fp8<T, 2>(fp, stream);
+    case 4: return launch_decode_fp8<T, 4>(fp, stream);
+    case 8: return launch_decode_fp8<T, 8>(fp, stream);
+    default: return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode_fp8: group %d", g);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status kv_write_fp8(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
+                        const int64_t *slot_mapping, int32_t num_tokens, const float *k_scale,
+                        const float *v_scale, void *k_pool, void *v_pool, void *stream) {
+    const char *fn = "kv_write_fp8";
+    pkv_status st = check_pool_desc(desc, fn);
+    if (st) return st;
+    if (desc->dtype == PKV_FP8_E4M3)
+        return fail(PKV_ERR_INVALID, "%s: desc->dtype is the type of the new values", fn);
+    if (desc->head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: only head_dim 128 is built", fn);
+    if (num_tokens < 0) return fail(PKV_ERR_INVALID, "%s: num_tokens < 0", fn);
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !slot_mapping || !k_scale || !v_scale || !k_pool || !v_pool)
+        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8) ||
+        !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(k_pool, 16) ||
+        !aligned(v_pool, 16))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    pkv::KvWriteFp8Params prm;
+    prm.k_new = k_new;
+    prm.v_new = v_new;
+    prm.slot_mapping = slot_mapping;
+    prm.k_scale = k_scale;
+    prm.v_scale = v_scale;
+    prm.k_pool = static_cast<uint8_t *>(k_pool);
+    prm.v_pool = static_cast<uint8_t *>(v_pool);
+    prm.T = num_tokens;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.D = desc->head_dim;
+    const int64_t total = (int64_t)num_tokens * prm.Hkv * (prm.D / 2);
+    const int64_t blocks = (total + 255) / 256;
+    if (blocks > INT_MAX) return fail(PKV_ERR_INVALID, "%s: too many tokens", fn);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    switch (desc->dtype) {
+    case PKV_F32: pkv::kv_write_fp8_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(prm); break;
+    case PKV_F16: pkv::kv_write_fp8_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(prm); break;
+    default:
+        pkv::kv_write_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(prm);
+        break;
+    }
+    return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+pkv_status paged_attn_decode_fp8(const pkv_attn_desc *desc, const void *q, const void *k_pool,
+                                 const void *v_pool, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables,
+                                 const int32_t *context_lens, float scale, void *out,
+                                 void *workspace, size_t workspace_bytes_given, void *stream) {
+    const char *fn = "paged_attn_decode_fp8";
+    Split sp;
+    pkv_status st = check_attn_desc(desc, fn, &sp);
+    if (st) return st;
+    if (desc->dtype != PKV_F16 && desc->dtype != PKV_BF16)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: q/out must be f16 or bf16", fn);
+    if (desc->head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: only head_dim 128 is built", fn);
+    if ((int64_t)desc->num_blocks * desc->num_kv_heads * pkv::kBlock >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_UNSUPPORTED, "%s: pool too large for 32-bit TMA rows", fn);
+    if (desc->num_seqs == 0) return PKV_OK;
+    if (!q || !k_pool || !v_pool || !k_scale || !v_scale || !block_tables || !context_lens ||
+        !out)
+        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
+    if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
+        !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_tables, 4) ||
+        !aligned(context_lens, 4))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID, "%s: scale is not finite", fn);
+    const size_t need = workspace_bytes(desc, sp);
+    if (need) {
+        if (!workspace || workspace_bytes_given < need)
+            return fail(PKV_ERR_INVALID, "%s: workspace needs %zu bytes", fn, need);
+        if (!aligned(workspace, 256))
+            return fail(PKV_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+    }
+    pkv::DecodeFp8Params fp;
+    pkv::DecodeParams &prm = fp.base;
+    prm.q = q;
+    prm.k_pool = k_pool;
+    prm.v_pool = v_pool;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.out = out;
+    const size_t rows = (size_t)desc->num_seqs * desc->num_q_heads * sp.pmax;
+    prm.ws_o = need ? static_cast<float *>(workspace) : nullptr;
+    prm.ws_ml = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 round_up(rows * desc->head_dim * 4, 256))
+                     : nullptr;
+    prm.S = desc->num_seqs;
+    prm.Hq = desc->num_q_heads;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.maxB = desc->max_blocks_per_seq;
+    prm.part_blocks = sp.part_blocks;
+    prm.pmax = sp.pmax;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    fp.k_scale = k_scale;
+    fp.v_scale = v_scale;
+    const int g = desc->num_q_heads / desc->num_kv_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (desc->dtype == PKV_F16) return dispatch_fp8<__half>(g, fp, s);
+    return dispatch_fp8<__nv_bfloat16>(g, fp, s);
 }
 
 }  // extern "C"

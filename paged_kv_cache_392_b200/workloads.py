@@ -194,3 +194,37 @@ def to_numpy_bits(t):
     if t.dtype == torch.float32:
         return t.numpy()
     return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def fp8_scales(wl, which):
+    """Per-kv-head scales for the FP8 cache: about 4.5 standard deviations map to the
+    largest E4M3 code (448), slightly different per head."""
+    h = np.arange(wl.num_kv_heads, dtype=np.float32)
+    base = np.float32(wl.kv_std * 4.5 / 448.0) * (np.float32(1.0) + np.float32(0.05) * h)
+    return base * (np.float32(1.0) if which == "k" else np.float32(1.1))
+
+
+def make_values_fp8(wl, device="cpu", torch=None):
+    """Inputs for an FP8 KV cache: q and new K/V as for ``make_values`` (in wl.dtype); the
+    pools as random E4M3 codes of N(0, kv_std^2) values at the per-head scales,
+    K [NB, Hkv, 16, D] and V [NB, Hkv, D, 16]; scales as fp32 tensors."""
+    if torch is None:
+        import torch  # noqa: F811
+    vals = make_values(wl, device, torch)
+    NB, Hkv, D = wl.num_blocks, wl.num_kv_heads, wl.head_dim
+    base = wl.seed * 1000003
+    ks = torch.from_numpy(fp8_scales(wl, "k")).to(device)
+    vs = torch.from_numpy(fp8_scales(wl, "v")).to(device)
+
+    def codes(shape, scale, seed, head_axis):
+        x = randn(torch, shape, "f32", wl.kv_std, seed, device)
+        view = [1] * len(shape)
+        view[head_axis] = -1
+        x = (x / scale.view(view)).clamp(-448.0, 448.0)
+        return x.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+
+    vals["k_pool"] = codes((NB, Hkv, wl.block_size, D), ks, base + 6, 1)
+    vals["v_pool"] = codes((NB, Hkv, D, wl.block_size), vs, base + 7, 1)
+    vals["k_scale"] = ks
+    vals["v_scale"] = vs
+    return vals

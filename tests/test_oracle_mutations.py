@@ -13,6 +13,7 @@ import pytest
 import oracle
 from oracle import build as obuild
 import tests.test_oracle_pins as pins
+import tests.test_oracle_pins_fp8 as pins8
 
 MUTATIONS = {
     "block index uses modulo": ("int64_t p = bt[(size_t)s * maxB + t / B];\n        int o = t % B;\n        double acc",
@@ -30,6 +31,17 @@ MUTATIONS = {
     "merge weight dropped": ("den += c * l[p];", "den += l[p];"),
     "one token too many": ("for (int t = 0; t < L; ++t) {\n        int64_t p = bt[(size_t)s * maxB + t / B];\n        int o = t % B;\n        double acc",
                            "for (int t = 0; t < L + (L % B != 0); ++t) {\n        int64_t p = bt[(size_t)s * maxB + t / B];\n        int o = t % B;\n        double acc"),
+    "e4m3 exponent bias": ("v = ldexp((double)(8 + f), e - 10);",
+                           "v = ldexp((double)(8 + f), e - 9);"),
+    "e4m3 encoder truncates": ("int n = (int)nearbyint(a / ldexp(1.0, e - 3));",
+                               "int n = (int)floor(a / ldexp(1.0, e - 3));"),
+    "fp8 V written untransposed": (
+        "v_pool[(((size_t)blk * Hkv + h) * D + d) * B + orc_v_slot(off)] =",
+        "v_pool[(((size_t)blk * Hkv + h) * B + orc_v_slot(off)) * D + d] ="),
+    "fp8 V slot order ignored": ("if (2 * (p / 4) + p % 2 + 8 * ((p / 2) % 2) == t) return p;",
+                                 "if (p == t) return p;"),
+    "fp8 K scale dropped": ("(orc_e4m3_to_f64(k_pool[(((size_t)p * Hkv + hk) * B + t % B) * D + d]) * ks)",
+                            "(orc_e4m3_to_f64(k_pool[(((size_t)p * Hkv + hk) * B + t % B) * D + d]))"),
     "copy skips v pool": ("memmove((char *)v_pool + (size_t)dst * blk_bytes,",
                           "if (0) memmove((char *)v_pool + (size_t)dst * blk_bytes,"),
 }
@@ -48,6 +60,10 @@ PINS = [
     lambda: pins.test_split_lse_merge_equals_one_pass(48),
     pins.test_kv_write_places_rows_at_their_slots_and_nothing_else,
     pins.test_kv_copy_blocks_copies_whole_blocks,
+    pins8.test_e4m3_decoder_matches_torch_for_all_codes,
+    pins8.test_e4m3_encoder_matches_torch_rounding_in_range,
+    pins8.test_kv_write_fp8_quantises_into_the_two_layouts,
+    pins8.test_fp8_decode_matches_bruteforce_on_dequantised_values,
 ]
 
 
