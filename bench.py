@@ -75,6 +75,9 @@ def parse_args(argv=None):
     ap.add_argument("--contiguous", action="store_true",
                     help="place each sequence's blocks contiguously and in order (paged "
                          "kernel over a contiguous layout) instead of shuffled")
+    ap.add_argument("--separate-write", action="store_true",
+                    help="kv_write and paged_attn_decode as two calls instead of the fused "
+                         "kv_write_and_decode (16-bit and fp32 caches)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
@@ -297,29 +300,32 @@ def hbm_peak():
 
 
 DECODE_SOURCES = ("attn_decode.cuh", "attn_decode_tc.cuh", "ptx.cuh", "faults.cuh")
+DECODE_FP8_SOURCES = DECODE_SOURCES + ("attn_decode_fp8.cuh", "pkv_cuda.cu")
 
 
-def kernel_source_sha():
-    """Hash of the decode kernels' sources (kernels and their launch shape)."""
+def kernel_source_sha(fp8=False):
+    """Hash of the decode kernels' sources (kernels and their launch shape); the FP8 kernel's
+    launch constants live in the launcher, so its hash covers that file too."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc")
-    for name in DECODE_SOURCES:
+    for name in (DECODE_FP8_SOURCES if fp8 else DECODE_SOURCES):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(workload):
+def profile_traffic(workload, fp8=False):
     """DRAM bytes per decode launch from the committed ncu summary for this workload, or
     None when there is none or it was taken on different kernel sources."""
-    path = os.path.join(ROOT, "profiles", "paged_attn_decode_%s.md" % workload)
+    path = os.path.join(ROOT, "profiles", "paged_attn_decode_%s%s.md"
+                        % ("fp8_" if fp8 else "", workload))
     try:
         text = open(path).read()
     except OSError:
         return None
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
-    if not m or not sha or sha.group(1) != kernel_source_sha():
+    if not m or not sha or sha.group(1) != kernel_source_sha(fp8):
         return None
     return float(m.group(1))
 
@@ -505,16 +511,23 @@ def run_pkv(args):
     rows_split, pmax = split_rows(wl, pt)
     nbytes = algorithmic_bytes(wl, pairs, rows_split, kv_es=1 if fp8 else None)
 
+    # 16-bit and fp32 caches take the newest token's write inside the decode kernel
+    # (kv_write_and_decode) unless --separate-write asks for the two calls.
+    fused = not fp8 and not args.separate_write
+
     def write(kn_, vn_, slots_):
         if fp8:
             B.kv_write_fp8(kn_, vn_, slots_, ksc, vsc, kp, vp)
-        else:
+        elif not fused:
             B.kv_write(kn_, vn_, slots_, kp, vp)
 
-    def decode(q_, bt_, lens_, out_):
+    def decode(q_, kn_, vn_, slots_, bt_, lens_, out_):
         if fp8:
             B.paged_attn_decode_fp8(q_, kp, vp, ksc, vsc, bt_, lens_, wl.scale, out=out_,
                                     workspace=ws, partition_tokens=pt)
+        elif fused:
+            B.kv_write_and_decode(q_, kn_, vn_, slots_, kp, vp, bt_, lens_, wl.scale,
+                                  out=out_, workspace=ws, partition_tokens=pt)
         else:
             B.paged_attn_decode(q_, kp, vp, bt_, lens_, wl.scale, out=out_, workspace=ws,
                                 partition_tokens=pt)
@@ -523,9 +536,10 @@ def run_pkv(args):
         if npairs:
             B.kv_copy_blocks(pairs_d, kp, vp)
         write(kn, vn, slots)
-        decode(q, bt, lens, out)
+        decode(q, kn, vn, slots, bt, lens, out)
 
-    launches_per_step = (1 if npairs else 0) + 1 + 1 + (1 if pmax > 1 else 0)
+    launches_per_step = (1 if npairs else 0) + (0 if fused else 1) + 1 + (1 if pmax > 1 else 0)
+    decode_call_bytes = nbytes["decode"] + (nbytes["kv_write"] if fused else 0)
 
     for _ in range(args.warmup):
         step()
@@ -552,7 +566,7 @@ def run_pkv(args):
                     B.kv_copy_blocks(pairs_d, kp, vp)
                 write(kn, vn, slots)
                 ev[j][0].record(gs)
-                decode(q, bt, lens, out)
+                decode(q, kn, vn, slots, bt, lens, out)
                 ev[j][1].record(gs)
         return g
 
@@ -610,7 +624,7 @@ def run_pkv(args):
         if npairs:
             B.kv_copy_blocks(d["pairs"], kp, vp)
         write(d["kn"], d["vn"], d["slots"])
-        decode(d["q"], d["bt"], d["lens"], outs[b])
+        decode(d["q"], d["kn"], d["vn"], d["slots"], d["bt"], d["lens"], outs[b])
 
     def h2d_copy(b, stream):
         with torch.cuda.stream(stream):
@@ -702,8 +716,8 @@ def run_pkv(args):
         peak, peak_kind = hbm_peak()
         step_ms = ms / K
         kv_gbs = world * nbytes["kv"] / (step_ms * 1e-3) / 1e9
-        achieved = nbytes["decode"] / (decode_ms * 1e-3) / 1e9
-        traffic = None if fp8 else profile_traffic(args.workload)
+        achieved = decode_call_bytes / (decode_ms * 1e-3) / 1e9
+        traffic = None if args.separate_write else profile_traffic(args.workload, fp8)
         probe = read_probe_gbs(torch, device) if args.read_probe else None
         swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe and not fp8 else None
         result = {
@@ -717,8 +731,8 @@ def run_pkv(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("f32 accumulate over fp8-e4m3 KV (codes widened to f16 for the "
-                      "tensor-core tiles), %s q/out" % wl.dtype) if fp8 else
+            "dtype": ("f32 accumulate over fp8-e4m3 KV (q.K on e4m3 tensor-core tiles, "
+                      "P.V on f16 tiles), %s q/out" % wl.dtype) if fp8 else
                      "f32 accumulate over %s KV" % wl.dtype,
             "data": "synthetic (seeded), no weights",
             "seqs_per_s": round(world * wl.num_seqs / (step_ms * 1e-3), 1),
@@ -736,10 +750,14 @@ def run_pkv(args):
                       (nbytes["kv"] / 1e9),
                 "parallelism": "replicas x%d" % world,
                 "placement": wl.extra.get("placement", "shuffled"),
+                "kv_write": ("kv_write_fp8 kernel" if fp8 else "fused into the decode kernel "
+                             "(kv_write_and_decode)" if fused else "separate kv_write kernel"),
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": "paged_attn_decode%s (decode + lse_reduce)" % ("_fp8" if fp8 else ""),
+                "kernel": ("paged_attn_decode_fp8 (decode + lse_reduce)" if fp8 else
+                           "kv_write_and_decode (newest-token write + decode, lse_reduce)"
+                           if fused else "paged_attn_decode (decode + lse_reduce)"),
                 "achieved": round(achieved, 1),
                 "peak": peak,
                 "peak_kind": peak_kind,
@@ -749,7 +767,7 @@ def run_pkv(args):
                 "read_probe_gbs": probe,
                 "frac_of_read_probe": round(achieved / probe, 4) if probe else None,
                 "traffic": traffic,
-                "algorithmic_bytes": nbytes["decode"],
+                "algorithmic_bytes": decode_call_bytes,
                 "avg_launch_ms": round(decode_ms, 5),
             },
             "e2e": {"value": round(world * nbytes["kv"] / (e2e_ms * 1e-3) / 1e9, 2),

@@ -123,6 +123,31 @@ pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_
                     void *v_pool, void *stream);
 
 /*
+ * One decode step in one launch: kv_write of each sequence's newest token followed by
+ * paged_attn_decode, with the write done inside the decode kernel ("Memory Optimization in
+ * LLM Serving with PagedAttention", section "How PagedAttention Works": the new token's
+ * K/V goes into its slot, then attention runs over the whole context).  The result equals
+ *     kv_write(desc, k_new, v_new, slot_mapping, num_seqs, k_pool, v_pool, stream);
+ *     paged_attn_decode(desc, q, k_pool, v_pool, block_tables, context_lens, scale, out,
+ *                       workspace, workspace_bytes, stream);
+ * bit for bit, under these conditions:
+ *   - token s of k_new / v_new ([S, H_kv, D] dtype, 16-byte aligned) belongs to sequence s,
+ *     and slot_mapping[s] (int64 [S], 8-byte aligned) is -1 (no write) or the slot of
+ *     position context_lens[s]-1, i.e. block_tables[s][(L-1)/16]*16 + (L-1)%16;
+ *   - the block holding that slot is read by no other sequence of the batch (copy-on-write
+ *     of shared blocks, kv_copy_blocks, must already have run; the block manager's
+ *     append_slot(s) guarantees this).
+ * A slot that is neither -1 nor the slot of position L-1 is not written and sets
+ * PKV_FAULT_BAD_SLOT.  Other arguments, errors and the workspace are as paged_attn_decode's.
+ * FP8 pools are rejected (PKV_ERR_INVALID).
+ */
+pkv_status kv_write_and_decode(const pkv_attn_desc *desc, const void *q, const void *k_new,
+                               const void *v_new, const int64_t *slot_mapping, void *k_pool,
+                               void *v_pool, const int32_t *block_tables,
+                               const int32_t *context_lens, float scale, void *out,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Copy-on-write block copy ("Memory Optimization in LLM Serving with PagedAttention",
  * section "Advanced Capabilities: Memory Sharing with Copy-on-Write": before a sequence
  * writes into a block it shares, the block's content is copied to a fresh block).  For each

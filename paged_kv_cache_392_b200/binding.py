@@ -31,6 +31,7 @@ EXPORTS = [
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
     "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
+    "kv_write_and_decode",
 ]
 
 
@@ -72,6 +73,8 @@ def lib():
         "paged_attn_decode": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz, vp], i32),
         "paged_attn_decode_no_alloc": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
         "kv_write": ([dp, vp, vp, vp, i32, vp, vp, vp], i32),
+        "kv_write_and_decode": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
+                                 sz, vp], i32),
         "kv_copy_blocks": ([dp, vp, i32, vp, vp, vp], i32),
         "pkv_device_faults": ([P(ctypes.c_uint32), ctypes.c_int, vp], i32),
         "pkv_bm_create": ([i32, i32, vp, P(vp)], i32),
@@ -205,6 +208,46 @@ def paged_attn_decode(q, k_pool, v_pool, block_tables, context_lens, scale, out=
                                    _ptr(block_tables), _ptr(context_lens), float(scale),
                                    _ptr(out), _ptr(workspace), nbytes,
                                    _stream(stream, q.device)))
+    return out
+
+
+def kv_write_and_decode(q, k_new, v_new, slot_mapping, k_pool, v_pool, block_tables,
+                        context_lens, scale, out=None, workspace=None, partition_tokens=0,
+                        stream=None):
+    """kv_write of each sequence's newest token (k_new / v_new [S, H_kv, D], slot_mapping
+    int64 [S]: -1 or the slot of position context_lens[s]-1) and paged_attn_decode, in one
+    launch.  Same result as the two calls when the slots' blocks are private to their
+    sequences."""
+    _dev(q, "q", k_pool.dtype)
+    _dev(k_new, "k_new", k_pool.dtype)
+    _dev(v_new, "v_new", k_pool.dtype)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    if q.dim() != 3 or block_tables.dim() != 2 or block_tables.shape[0] != q.shape[0] or \
+            context_lens.shape != (q.shape[0],):
+        raise ValueError("q [S,Hq,D], block_tables [S,maxB], context_lens [S] expected")
+    desc = decode_desc(q, k_pool, v_pool, block_tables, partition_tokens)
+    if q.shape[2] != k_pool.shape[3]:
+        raise ValueError("head_dim mismatch")
+    if k_new.shape != (q.shape[0], k_pool.shape[1], q.shape[2]) or v_new.shape != k_new.shape \
+            or slot_mapping.shape != (q.shape[0],):
+        raise ValueError("k_new / v_new [S, H_kv, D] and slot_mapping [S] expected")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _dev(out, "out", q.dtype)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    need = attn_workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().kv_write_and_decode(ctypes.byref(desc), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                     _ptr(slot_mapping), _ptr(k_pool), _ptr(v_pool),
+                                     _ptr(block_tables), _ptr(context_lens), float(scale),
+                                     _ptr(out), _ptr(workspace), nbytes,
+                                     _stream(stream, q.device)))
     return out
 
 

@@ -42,6 +42,12 @@ namespace pkv {
 constexpr int kDefaultPartitionTokens = 512;
 
 constexpr int kBlock = 16;                       // tokens per KV block
+// Lazy online-softmax rescale threshold (base-2 logit units): a running max moves only when
+// a block's max exceeds it by more than this, so exponents stay <= 2^8.
+#ifndef PKV_LAZY_RESCALE
+#define PKV_LAZY_RESCALE 8
+#endif
+constexpr float kLazyRescale = float(PKV_LAZY_RESCALE);
 constexpr uint64_t kWaitTimeoutNs = 1000000000;  // bounded shared-memory barrier waits (1 s)
 
 
@@ -58,7 +64,45 @@ struct DecodeParams {
     int32_t part_blocks;  // blocks per partition
     int32_t pmax;         // partitions of the longest admissible sequence
     float scale_log2;     // scale * log2(e)
+    // fused kv_write (NULL: none): token s of k_new / v_new [S][H_kv][D] is sequence s's
+    // newest token, stored into slot_mapping[s] before the decode reads it
+    const void *k_new = nullptr;
+    const void *v_new = nullptr;
+    const int64_t *slot_mapping = nullptr;
 };
+
+// Fused kv_write, called by the one warp per (sequence, kv head) that will copy the block
+// holding position L-1.  The warp stores the newest token's K and V rows of kv head hk into
+// their slot, then fences its generic-proxy stores against its own later bulk / TMA copies
+// (async proxy) of that block.  A slot of -1 is skipped; a slot other than the one of
+// position L-1 is not written and sets fault bit 4 (bad slot).
+template <typename T, int D>
+__device__ __forceinline__ void write_newest_token(const DecodeParams &p, int s, int hk, int L,
+                                                   int lane) {
+    const int64_t slot = p.slot_mapping[s];
+    if (slot != -1) {
+        const int32_t blk = p.block_tables[(size_t)s * p.maxB + (L - 1) / kBlock];
+        const int off = (L - 1) % kBlock;
+        if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
+            constexpr int VPR = D * (int)sizeof(T) / 16;  // 16-byte vectors per row
+            const size_t src = ((size_t)s * p.Hkv + hk) * VPR;
+            const size_t dst = (((size_t)blk * p.Hkv + hk) * kBlock + off) * VPR;
+            // the pools are written only here; the decode itself reads them
+            uint4 *kp = static_cast<uint4 *>(const_cast<void *>(p.k_pool));
+            uint4 *vp = static_cast<uint4 *>(const_cast<void *>(p.v_pool));
+            for (int v = lane; v < 2 * VPR; v += 32) {
+                if (v < VPR)
+                    kp[dst + v] = static_cast<const uint4 *>(p.k_new)[src + v];
+                else
+                    vp[dst + v - VPR] = static_cast<const uint4 *>(p.v_new)[src + v - VPR];
+            }
+            fence_proxy_async_global();
+        } else if (lane == 0) {
+            atomicOr(&g_faults, (unsigned)blk < (unsigned)p.NB ? 0x4u : 0x2u);
+        }
+    }
+    __syncwarp();
+}
 
 // ---- element conversions --------------------------------------------------------------
 template <typename T>
@@ -259,6 +303,8 @@ paged_attn_decode_kernel(const DecodeParams p) {
         fence_mbar_init();
     }
     __syncwarp();
+    if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
+        write_newest_token<T, D>(p, s, hk, L, lane);
 
     const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
     const char *kbase = static_cast<const char *>(p.k_pool);

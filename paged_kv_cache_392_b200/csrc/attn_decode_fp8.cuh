@@ -30,10 +30,14 @@ __host__ __device__ __forceinline__ int v_slot_of_token(int t) {
     return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
 }
 
-// Two E4M3 codes (low byte first) to an f16x2 register, exactly.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Two E4M3 codes (bytes 0 and 1 of w) to an f16x2 register holding each value times 2^-8,
+// with integer operations only: an E4M3 code s.eeee.mmm placed as the f16 s.0eeee.mmm0000000
+// is the same number scaled by 2^(7-15) = 2^-8, subnormals included (f16 keeps E4M3's
+// subnormal grid scaled by the same power of two).  byte << 8 puts s.eeee.mmm at bits
+// 15..8; subtracting ((x >> 1) & 0x3F80) moves eeee.mmm down one bit and keeps s.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
+    const uint32_t t = __byte_perm(w, 0u, sel);  // [b_hi : 0 : b_lo : 0]
+    return t - ((t >> 1) & 0x3F803F80u);
 }
 
 // D = A * B + C for one m16n8k32 tile of E4M3 codes, fp32 accumulators.
@@ -65,13 +69,21 @@ struct DecodeFp8Cfg {
     static constexpr int RING = W * NSW * STAGE;
     static constexpr int BARS = W * NSW * 8;
     static constexpr int KSTEPS = D / 16;
+    // the warps' merge states [W][G][D] + [W][G][2] floats reuse the ring once every warp
+    // is done with it
     template <int G>
-    static constexpr int smem() { return 1024 + RING + BARS + W * G * (D + 2) * 4; }
+    static constexpr int smem() {
+        static_assert(W * G * (D + 2) * 4 <= RING, "merge states must fit in the ring");
+        return 1024 + RING + BARS;
+    }
 };
 
 // T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.
+// Resident warps per SM the register budget is sized for (16: 128 registers a thread).
+constexpr int kFp8WarpsPerSm = 16;
+
 template <typename T, int G, int W, int NSW>
-__global__ void __launch_bounds__(W * 32)
+__global__ void __launch_bounds__(W * 32, kFp8WarpsPerSm / W)
 paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                              const DecodeFp8Params fp) {
     using C = DecodeFp8Cfg<W, NSW>;
@@ -110,7 +122,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
 
     unsigned char *ring = smem + warp * NSW * C::STAGE;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::RING) + warp * NSW;
-    float *mo = reinterpret_cast<float *>(smem + C::RING + C::BARS);
+    float *mo = reinterpret_cast<float *>(smem);  // over the ring, after the block loop
     float *mml = mo + W * G * D;
 
     if (lane == 0) {
@@ -201,8 +213,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                     const float2 x = make_float2(qv[j][b][e] * qf_mine, qv[j][b][e + 1] * qf_mine);
                     const __nv_fp8x2_storage_t h2 = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
                     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h2, __NV_E4M3);
-                    const float2 r = make_float2(x.x - __half2float(__half(hr.x)),
-                                                 x.y - __half2float(__half(hr.y)));
+                    const float2 r = make_float2(x.x - __half2float(__ushort_as_half(hr.x)),
+                                                 x.y - __half2float(__ushort_as_half(hr.y)));
                     const __nv_fp8x2_storage_t l2 = __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
                     hi |= static_cast<uint32_t>(h2) << (8 * e);
                     lo |= static_cast<uint32_t>(l2) << (8 * e);
@@ -267,7 +279,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
 
         // ---- S^T = K Q^T on E4M3 tiles: K codes go from ldmatrix straight into the A
         // fragments (row g / g+8, k 4tq..4tq+3 and 16+4tq..16+4tq+3 of each 32-dim step)
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        // the high and residual q terms accumulate separately: two MMA chains of K32
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sres[4] = {0.f, 0.f, 0.f, 0.f};
         const uint32_t kb = smem_u32(Ks);
 #pragma unroll
         for (int j = 0; j < K32; ++j) {
@@ -275,8 +288,10 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             uint32_t a[4];
             ldmatrix_x4(a, kb + k_tok * 128 + ((c ^ (k_tok & 7)) << 4));
             mma_16832_e4m3(sacc, a, qhi[j][0], qhi[j][1]);
-            mma_16832_e4m3(sacc, a, qlo[j][0], qlo[j][1]);
+            mma_16832_e4m3(sres, a, qlo[j][0], qlo[j][1]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
 
         // ---- online softmax (lane: tokens g, g+8 of heads 2tq, 2tq+1) --------------------
         const float x0 = g < nvalid ? sacc[0] * sl0 : -INFINITY;
@@ -289,10 +304,15 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
             bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
         }
-        const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
+        // Lazy rescale: the reference max moves only when a block's max passes it by more
+        // than kLazyRescale (base 2), so P stays <= 2^kLazyRescale (f16 holds it) and most
+        // blocks skip the rescale of O; O / l is unchanged by the choice of reference.
+        const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
+        const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
         const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
         const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-        const float a0 = exp2f(m_run[0] - mn0), a1 = exp2f(m_run[1] - mn1);
+        const float a0 = mn0 == m_run[0] ? 1.f : exp2f(m_run[0] - mn0);
+        const float a1 = mn1 == m_run[1] ? 1.f : exp2f(m_run[1] - mn1);
         float s0 = p0 + p2, s1 = p1 + p3;
 #pragma unroll
         for (int m = 4; m < 32; m <<= 1) {
@@ -327,12 +347,12 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             ldmatrix_x4(r, vb + (32 * t2 + v_row) * 16);
             // r[0]: dims 32t2+0..7, r[1]: +8..15 (m-tile 2t2); r[2], r[3]: m-tile 2t2+1
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < 2; ++h) {  // V x 2^-8 widened to f16 on the integer pipe
                 uint32_t a[4];
-                a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] & 0xffffu));
-                a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] >> 16));
-                a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] & 0xffffu));
-                a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] >> 16));
+                a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x1404u);
+                a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x3424u);
+                a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x1404u);
+                a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x3424u);
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }
         }
@@ -354,7 +374,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
     }
 
-    const float vsc = fp.v_scale[hk];
+    __syncthreads();  // every warp is done with its ring: the merge states go over it
+    const float vsc = fp.v_scale[hk] * 256.f;  // the integer widening scaled V by 2^-8
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
     if (h0 < G) {
         float *dst = mo + (warp * G + h0) * D;

@@ -104,6 +104,8 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
         }
     }
     __syncwarp();
+    if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
+        write_newest_token<T, D>(p, s, hk, L, lane);
 
     const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
     const uint64_t policy = l2_evict_first_policy();
@@ -220,10 +222,13 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
             bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
             bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
         }
-        const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
+        // lazy rescale: the reference max moves only past a margin of kLazyRescale
+        const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
+        const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
         const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
         const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-        const float a0 = exp2f(m_run[0] - mn0), a1 = exp2f(m_run[1] - mn1);
+        const float a0 = mn0 == m_run[0] ? 1.f : exp2f(m_run[0] - mn0);
+        const float a1 = mn1 == m_run[1] ? 1.f : exp2f(m_run[1] - mn1);
         float s0 = p0 + p2, s1 = p1 + p3;
 #pragma unroll
         for (int m = 4; m < 32; m <<= 1) {

@@ -125,3 +125,72 @@ def test_random_traffic_invariants():
         # only the last block of a sequence is partly empty
         for s in live:
             assert 0 <= bm.waste(s) < 16 or bm.seq_len(s) == 0
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_swap_fork_cow_traffic_keeps_every_sequence_readable(seed):
+    """Data-level pin of fork, copy-on-write and swap: device and host memory are simulated
+    cell by cell, the model's copy pairs and slots are applied as a caller would, and every
+    live sequence must read back exactly the tokens it holds, through its own table, from
+    the pool it lives in."""
+    rng = np.random.default_rng(300 + seed)
+    NB, NH, B = 40, 30, 16
+    bm = BlockManagerModel(NB, B, free_order=rng.permutation(NB))
+    bm.set_host_pool(NH, rng.permutation(NH))
+    dev = [[None] * B for _ in range(NB)]
+    host = [[None] * B for _ in range(NH)]
+    want, nxt = {}, 0          # seq -> list of token labels it holds
+
+    def write(seq, slot):
+        dev[slot // B][slot % B] = (seq, len(want[seq]))
+        want[seq].append((seq, len(want[seq])))
+
+    for _ in range(2500):
+        live = list(want)
+        on_gpu = [s for s in live if not bm.is_swapped(s)]
+        off = [s for s in live if bm.is_swapped(s)]
+        op = int(rng.integers(0, 10))
+        try:
+            if op == 0 or not live:
+                n = int(rng.integers(0, 50))
+                bm.add_seq(nxt, n)
+                want[nxt] = []
+                tbl = bm.block_table(nxt)
+                for t in range(n):
+                    write(nxt, tbl[t // B] * B + t % B)
+                nxt += 1
+            elif op == 1 and on_gpu:
+                p = on_gpu[int(rng.integers(len(on_gpu)))]
+                bm.fork(p, nxt)
+                want[nxt] = list(want[p])
+                nxt += 1
+            elif op == 2:
+                s = live[int(rng.integers(len(live)))]
+                bm.free_seq(s)
+                del want[s]
+            elif op == 3 and on_gpu:
+                s = on_gpu[int(rng.integers(len(on_gpu)))]
+                for g, h in bm.swap_out(s):
+                    host[h] = list(dev[g])
+            elif op == 4 and off:
+                s = off[int(rng.integers(len(off)))]
+                for h, g in bm.swap_in(s):
+                    dev[g] = list(host[h])
+            elif on_gpu:
+                s = on_gpu[int(rng.integers(len(on_gpu)))]
+                slot, cow = bm.append_slot(s)
+                if cow is not None:
+                    dev[cow[1]] = list(dev[cow[0]])
+                write(s, slot)
+        except OutOfBlocks:
+            s = live[0]
+            bm.free_seq(s)
+            del want[s]
+        for s, toks in want.items():
+            mem = host if bm.is_swapped(s) else dev
+            tbl = bm.block_table(s)
+            assert bm.seq_len(s) == len(toks)
+            assert [mem[tbl[t // B]][t % B] for t in range(len(toks))] == toks
+        # host blocks are never shared: each belongs to one swapped sequence or is free
+        held = [h for s in want if bm.is_swapped(s) for h in bm.block_table(s)]
+        assert sorted(held + list(bm.host_free_order())) == list(range(NH))

@@ -1,0 +1,106 @@
+"""GPU: kv_write_and_decode, the newest token's kv_write done inside the decode kernel,
+against the oracle's kv_write followed by its decode, and bit for bit against the two
+separate calls on the same inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_392_b200 import binding as B
+from paged_kv_cache_392_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "f16": 2e-3, "bf16": 1e-2}
+RAGGED = [1, 2, 15, 16, 17, 31, 33, 100, 255, 256, 257, 511, 512, 513, 700, 1024, 1500]
+
+
+@pytest.fixture(autouse=True)
+def _clean_faults():
+    B.device_faults(clear=True)
+    yield
+    assert B.device_faults(clear=True) == []
+
+
+def bits(t):
+    return W.to_numpy_bits(t)
+
+
+def fused_and_separate(wl, vals, slots, pt):
+    """Run the fused call on one copy of the pools and kv_write + paged_attn_decode on
+    another; return (out_fused, out_separate, pools_fused, pools_separate)."""
+    d = {k: v.cuda() for k, v in vals.items()}
+    kp2, vp2 = d["k_pool"].clone(), d["v_pool"].clone()
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    sl = torch.from_numpy(slots).cuda()
+    out1 = B.kv_write_and_decode(d["q"], d["k_new"], d["v_new"], sl, d["k_pool"], d["v_pool"],
+                                 bt, lens, wl.scale, partition_tokens=pt)
+    B.kv_write(d["k_new"], d["v_new"], sl, kp2, vp2)
+    out2 = B.paged_attn_decode(d["q"], kp2, vp2, bt, lens, wl.scale, partition_tokens=pt)
+    torch.cuda.synchronize()
+    return out1, out2, (d["k_pool"], d["v_pool"]), (kp2, vp2)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2)])
+@pytest.mark.parametrize("pt", [0, 64])
+def test_fused_step_matches_oracle_and_separate_calls(dtype, Hq, Hkv, pt):
+    D = 64 if dtype == "f32" else 128
+    wl = W.make_workload("fused", RAGGED, Hq, Hkv, D, dtype, 31 * Hq + Hkv + pt,
+                         pool_factor=1.3, partition_tokens=pt)
+    if dtype == "f32":
+        wl.kv_std = 1.0
+    vals = W.make_values(wl, "cpu")
+    out1, out2, (kp1, vp1), (kp2, vp2) = fused_and_separate(wl, vals, wl.slot_mapping, pt)
+    assert np.array_equal(bits(kp1), bits(kp2)) and np.array_equal(bits(vp1), bits(vp2))
+    assert np.array_equal(bits(out1), bits(out2))
+    kp, vp = bits(vals["k_pool"]).copy(), bits(vals["v_pool"]).copy()
+    oracle.kv_write(bits(vals["k_new"]), bits(vals["v_new"]), wl.slot_mapping, kp, vp)
+    assert np.array_equal(bits(kp1), kp) and np.array_equal(bits(vp1), vp)
+    ref = oracle.paged_attn_decode(bits(vals["q"]), kp, vp, wl.block_tables, wl.context_lens,
+                                   wl.scale, dtype)
+    err = np.max(np.abs(out1.double().cpu().numpy() - ref))
+    assert err <= TOL[dtype], err
+
+
+def test_fused_skips_minus_one_slots():
+    wl = W.make_workload("skip", RAGGED, 8, 2, 128, "bf16", 5, pool_factor=1.3)
+    vals = W.make_values(wl, "cpu")
+    slots = wl.slot_mapping.copy()
+    slots[::3] = -1
+    out1, out2, (kp1, vp1), (kp2, vp2) = fused_and_separate(wl, vals, slots, 0)
+    assert np.array_equal(bits(kp1), bits(kp2)) and np.array_equal(bits(vp1), bits(vp2))
+    assert np.array_equal(bits(out1), bits(out2))
+    kp, vp = bits(vals["k_pool"]).copy(), bits(vals["v_pool"]).copy()
+    oracle.kv_write(bits(vals["k_new"]), bits(vals["v_new"]), slots, kp, vp)
+    assert np.array_equal(bits(kp1), kp) and np.array_equal(bits(vp1), vp)
+
+
+def test_fused_refuses_a_slot_that_is_not_the_newest_position():
+    wl = W.make_workload("bad", [20, 40, 33], 4, 4, 64, "f16", 6, pool_factor=1.5)
+    vals = {k: v.cuda() for k, v in W.make_values(wl, "cpu").items()}
+    kp0, vp0 = vals["k_pool"].clone(), vals["v_pool"].clone()
+    slots = wl.slot_mapping.copy()
+    slots[1] -= 1                       # position L-2 of sequence 1: not the newest token
+    out = B.kv_write_and_decode(vals["q"], vals["k_new"], vals["v_new"],
+                                torch.from_numpy(slots).cuda(), vals["k_pool"],
+                                vals["v_pool"], torch.from_numpy(wl.block_tables).cuda(),
+                                torch.from_numpy(wl.context_lens).cuda(), wl.scale)
+    assert B.device_faults() == ["bad slot"]
+    # sequences 0 and 2 were written, sequence 1 was not
+    kp_ref, vp_ref = kp0.clone(), vp0.clone()
+    for s in (0, 2):
+        sl = int(wl.slot_mapping[s])
+        kp_ref[sl // 16, :, sl % 16] = vals["k_new"][s]
+        vp_ref[sl // 16, :, sl % 16] = vals["v_new"][s]
+    assert torch.equal(vals["k_pool"], kp_ref) and torch.equal(vals["v_pool"], vp_ref)
+    assert torch.isfinite(out).all()
+
+
+def test_fused_full_size_gqa_matches_separate_calls():
+    wl = W.gqa()
+    vals = W.make_values(wl, "cuda")
+    out1, out2, (kp1, vp1), (kp2, vp2) = fused_and_separate(wl, vals, wl.slot_mapping, 0)
+    assert torch.equal(kp1, kp2) and torch.equal(vp1, vp2)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
