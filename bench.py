@@ -76,8 +76,8 @@ def parse_args(argv=None):
                     help="place each sequence's blocks contiguously and in order (paged "
                          "kernel over a contiguous layout) instead of shuffled")
     ap.add_argument("--separate-write", action="store_true",
-                    help="kv_write and paged_attn_decode as two calls instead of the fused "
-                         "kv_write_and_decode (16-bit and fp32 caches)")
+                    help="the newest token's write as its own kernel (kv_write / "
+                         "kv_write_fp8) before the decode, instead of the fused call")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
@@ -511,18 +511,23 @@ def run_pkv(args):
     rows_split, pmax = split_rows(wl, pt)
     nbytes = algorithmic_bytes(wl, pairs, rows_split, kv_es=1 if fp8 else None)
 
-    # 16-bit and fp32 caches take the newest token's write inside the decode kernel
-    # (kv_write_and_decode) unless --separate-write asks for the two calls.
-    fused = not fp8 and not args.separate_write
+    # The newest token's write runs inside the decode kernel (kv_write_and_decode,
+    # kv_write_fp8_and_decode) unless --separate-write asks for the two calls.
+    fused = not args.separate_write
 
     def write(kn_, vn_, slots_):
+        if fused:
+            return
         if fp8:
             B.kv_write_fp8(kn_, vn_, slots_, ksc, vsc, kp, vp)
-        elif not fused:
+        else:
             B.kv_write(kn_, vn_, slots_, kp, vp)
 
     def decode(q_, kn_, vn_, slots_, bt_, lens_, out_):
-        if fp8:
+        if fp8 and fused:
+            B.kv_write_fp8_and_decode(q_, kn_, vn_, slots_, ksc, vsc, kp, vp, bt_, lens_,
+                                      wl.scale, out=out_, workspace=ws, partition_tokens=pt)
+        elif fp8:
             B.paged_attn_decode_fp8(q_, kp, vp, ksc, vsc, bt_, lens_, wl.scale, out=out_,
                                     workspace=ws, partition_tokens=pt)
         elif fused:
@@ -750,14 +755,16 @@ def run_pkv(args):
                       (nbytes["kv"] / 1e9),
                 "parallelism": "replicas x%d" % world,
                 "placement": wl.extra.get("placement", "shuffled"),
-                "kv_write": ("kv_write_fp8 kernel" if fp8 else "fused into the decode kernel "
-                             "(kv_write_and_decode)" if fused else "separate kv_write kernel"),
+                "kv_write": ("fused into the decode kernel" if fused else
+                             "separate %s kernel" % ("kv_write_fp8" if fp8 else "kv_write")),
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": ("paged_attn_decode_fp8 (decode + lse_reduce)" if fp8 else
-                           "kv_write_and_decode (newest-token write + decode, lse_reduce)"
-                           if fused else "paged_attn_decode (decode + lse_reduce)"),
+                "kernel": "%s (%sdecode + lse_reduce)" % (
+                    {(True, True): "kv_write_fp8_and_decode", (True, False):
+                     "paged_attn_decode_fp8", (False, True): "kv_write_and_decode",
+                     (False, False): "paged_attn_decode"}[(fp8, fused)],
+                    "newest-token write + " if fused else ""),
                 "achieved": round(achieved, 1),
                 "peak": peak,
                 "peak_kind": peak_kind,

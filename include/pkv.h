@@ -52,7 +52,9 @@ typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_FP8_E4M3 = 
 /* Bits of the device fault word. */
 #define PKV_FAULT_BAD_LEN   0x1u  /* context_lens[s] outside [1, max_blocks_per_seq*16]  */
 #define PKV_FAULT_BAD_BLOCK 0x2u  /* block table entry outside [0, num_blocks)          */
-#define PKV_FAULT_BAD_SLOT  0x4u  /* slot outside [0, num_blocks*16) and not -1         */
+#define PKV_FAULT_BAD_SLOT  0x4u  /* slot outside [0, num_blocks*16) and not -1; in the  */
+                                  /* fused write-and-decode calls, a slot that is not    */
+                                  /* -1 and not the one of position context_lens[s]-1    */
 #define PKV_FAULT_BAD_PAIR  0x8u  /* copy pair naming a block outside [0, num_blocks)   */
 #define PKV_FAULT_TIMEOUT   0x10u /* a bounded wait on a shared-memory barrier gave up  */
 
@@ -209,6 +211,22 @@ pkv_status paged_attn_decode_fp8(const pkv_attn_desc *desc, const void *q, const
                                  const float *v_scale, const int32_t *block_tables,
                                  const int32_t *context_lens, float scale, void *out,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * kv_write_fp8 of each sequence's newest token fused into paged_attn_decode_fp8 (one launch),
+ * as kv_write_and_decode is for 16-bit pools: token s of k_new / v_new ([S, H_kv, D] of
+ * desc->dtype, 16-byte aligned) is quantised into slot_mapping[s] (int64 [S]), which must be
+ * -1 or the slot of position context_lens[s]-1 in a block no other sequence of the batch
+ * reads.  The pools then hold exactly what kv_write_fp8 writes and the output equals
+ * paged_attn_decode_fp8's on those pools, bit for bit.  A slot other than -1 or position
+ * L-1's is not written and sets PKV_FAULT_BAD_SLOT.
+ */
+pkv_status kv_write_fp8_and_decode(const pkv_attn_desc *desc, const void *q, const void *k_new,
+                                   const void *v_new, const int64_t *slot_mapping,
+                                   const float *k_scale, const float *v_scale, void *k_pool,
+                                   void *v_pool, const int32_t *block_tables,
+                                   const int32_t *context_lens, float scale, void *out,
+                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Allocation-free variant of paged_attn_decode.  The paper has no counterpart: this entry

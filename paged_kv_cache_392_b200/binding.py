@@ -31,7 +31,7 @@ EXPORTS = [
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
     "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
-    "kv_write_and_decode",
+    "kv_write_and_decode", "kv_write_fp8_and_decode",
 ]
 
 
@@ -101,6 +101,8 @@ def lib():
         "kv_write_fp8": ([dp, vp, vp, vp, i32, vp, vp, vp, vp, vp], i32),
         "paged_attn_decode_fp8": ([dp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz,
                                    vp], i32),
+        "kv_write_fp8_and_decode": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float,
+                                     vp, vp, sz, vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -382,6 +384,41 @@ def paged_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, block_tables, con
                                        _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
                                        _ptr(context_lens), float(scale), _ptr(out),
                                        _ptr(workspace), nbytes, _stream(stream, q.device)))
+    return out
+
+
+def kv_write_fp8_and_decode(q, k_new, v_new, slot_mapping, k_scale, v_scale, k_pool, v_pool,
+                            block_tables, context_lens, scale, out=None, workspace=None,
+                            partition_tokens=0, stream=None):
+    """kv_write_fp8 of each sequence's newest token (k_new / v_new [S, H_kv, D] in q's dtype,
+    slot_mapping int64 [S]: -1 or the slot of position context_lens[s]-1) fused into
+    paged_attn_decode_fp8: one launch, same pools and output as the two calls."""
+    NB, Hkv, Bs, D = _fp8_pools(k_pool, v_pool)
+    _dev(q, "q")
+    _dev(k_new, "k_new", q.dtype)
+    _dev(v_new, "v_new", q.dtype)
+    _dev(slot_mapping, "slot_mapping", torch.int64)
+    _dev(k_scale, "k_scale", torch.float32)
+    _dev(v_scale, "v_scale", torch.float32)
+    _dev(block_tables, "block_tables", torch.int32)
+    _dev(context_lens, "context_lens", torch.int32)
+    S, Hq, Dq = q.shape
+    if Dq != D or block_tables.shape[0] != S or context_lens.shape != (S,):
+        raise ValueError("q [S,Hq,D], block_tables [S,maxB], context_lens [S] expected")
+    if k_new.shape != (S, Hkv, D) or v_new.shape != k_new.shape or slot_mapping.shape != (S,):
+        raise ValueError("k_new / v_new [S, H_kv, D] and slot_mapping [S] expected")
+    desc = make_desc(S, Hq, Hkv, D, NB, block_tables.shape[1], q.dtype, partition_tokens, Bs)
+    if out is None:
+        out = torch.empty_like(q)
+    need = attn_workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().kv_write_fp8_and_decode(
+        ctypes.byref(desc), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping),
+        _ptr(k_scale), _ptr(v_scale), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
+        _ptr(context_lens), float(scale), _ptr(out), _ptr(workspace), nbytes,
+        _stream(stream, q.device)))
     return out
 
 

@@ -61,6 +61,61 @@ struct DecodeFp8Params {
     const float *v_scale;     // [H_kv]
 };
 
+template <typename T>
+__device__ __forceinline__ float load_elem(const void *base, int64_t i) {
+    if constexpr (std::is_same<T, float>::value)
+        return static_cast<const float *>(base)[i];
+    else if constexpr (std::is_same<T, __half>::value)
+        return __half2float(static_cast<const __half *>(base)[i]);
+    else
+        return __bfloat162float(static_cast<const __nv_bfloat16 *>(base)[i]);
+}
+
+// E4M3 codes of src[i] / scale and src[i+1] / scale (fp32 division, round to nearest even,
+// saturating to +-448), element i in the low byte: the cache format's quantisation.
+template <typename T>
+__device__ __forceinline__ __nv_fp8x2_storage_t quantize2(const void *src, int64_t i,
+                                                         float scale) {
+    const float2 x = make_float2(load_elem<T>(src, i) / scale, load_elem<T>(src, i + 1) / scale);
+    return __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Fused kv_write_fp8 of sequence s's newest token for kv head hk, by the one warp that will
+// copy the block holding position L-1: quantise the K row and the V column into their slot,
+// then fence the generic-proxy stores against the warp's own TMA / bulk copies of the block.
+// A slot of -1 is skipped; any slot other than position L-1's sets fault bit 4 (bad slot)
+// and is not written.
+template <typename T>
+__device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp, int s, int hk,
+                                                       int L, int lane) {
+    constexpr int D = 128;
+    const DecodeParams &p = fp.base;
+    const int64_t slot = p.slot_mapping[s];
+    if (slot != -1) {
+        const int32_t blk = p.block_tables[(size_t)s * p.maxB + (L - 1) / kBlock];
+        const int off = (L - 1) % kBlock;
+        if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
+            const int64_t src = ((int64_t)s * p.Hkv + hk) * D;
+            const int64_t hb = (int64_t)blk * p.Hkv + hk;
+            const int vs = v_slot_of_token(off);
+            // the pools are written only here; the decode itself reads them
+            uint8_t *kp = static_cast<uint8_t *>(const_cast<void *>(p.k_pool));
+            uint8_t *vp = static_cast<uint8_t *>(const_cast<void *>(p.v_pool));
+            for (int d = 2 * lane; d < D; d += 64) {
+                const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src + d, fp.k_scale[hk]);
+                const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src + d, fp.v_scale[hk]);
+                *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + (hb * kBlock + off) * D + d) = kc;
+                vp[(hb * D + d) * kBlock + vs] = static_cast<uint8_t>(vc & 0xffu);
+                vp[(hb * D + d + 1) * kBlock + vs] = static_cast<uint8_t>(vc >> 8);
+            }
+            fence_proxy_async_global();
+        } else if (lane == 0) {
+            atomicOr(&g_faults, (unsigned)blk < (unsigned)p.NB ? 0x4u : 0x2u);
+        }
+    }
+    __syncwarp();
+}
+
 template <int W, int NSW>
 struct DecodeFp8Cfg {
     static constexpr int D = 128;
@@ -132,6 +187,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         if (warp == 0) prefetch_tmap(&tmk);
     }
     __syncwarp();
+    if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
+        write_newest_token_fp8<T>(fp, s, hk, L, lane);
 
     const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
     const char *vbase = static_cast<const char *>(p.v_pool);
@@ -417,15 +474,6 @@ struct KvWriteFp8Params {
     int32_t T, Hkv, NB, D;
 };
 
-template <typename T>
-__device__ __forceinline__ float load_elem(const void *base, int64_t i) {
-    if constexpr (std::is_same<T, float>::value)
-        return static_cast<const float *>(base)[i];
-    else if constexpr (std::is_same<T, __half>::value)
-        return __half2float(static_cast<const __half *>(base)[i]);
-    else
-        return __bfloat162float(static_cast<const __nv_bfloat16 *>(base)[i]);
-}
 
 // One thread per (token, head, pair of dims): codes of x / scale, RNE, saturating.
 template <typename T>
@@ -446,13 +494,8 @@ __global__ void __launch_bounds__(256) kv_write_fp8_kernel(const KvWriteFp8Param
     const int64_t blk = slot >> 4;
     const int off = (int)(slot & 15);
     const int64_t src = th * p.D + d;
-    const float ks = p.k_scale[h], vs = p.v_scale[h];
-    const float2 kx = make_float2(load_elem<T>(p.k_new, src) / ks,
-                                  load_elem<T>(p.k_new, src + 1) / ks);
-    const float2 vx = make_float2(load_elem<T>(p.v_new, src) / vs,
-                                  load_elem<T>(p.v_new, src + 1) / vs);
-    const __nv_fp8x2_storage_t kc = __nv_cvt_float2_to_fp8x2(kx, __NV_SATFINITE, __NV_E4M3);
-    const __nv_fp8x2_storage_t vc = __nv_cvt_float2_to_fp8x2(vx, __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src, p.k_scale[h]);
+    const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src, p.v_scale[h]);
     const int64_t hb = blk * p.Hkv + h;
     *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + (hb * 16 + off) * p.D + d) = kc;
     const int sp = v_slot_of_token(off);

@@ -476,6 +476,71 @@ pkv_status dispatch_fp8(int g, const pkv::DecodeFp8Params &fp, cudaStream_t stre
     }
 }
 
+// Shared body of paged_attn_decode_fp8 and kv_write_fp8_and_decode (k_new / v_new /
+// slot_mapping NULL: no fused write).
+pkv_status decode_fp8_impl(const pkv_attn_desc *desc, const void *q, const void *k_new,
+                           const void *v_new, const int64_t *slot_mapping, const void *k_pool,
+                           const void *v_pool, const float *k_scale, const float *v_scale,
+                           const int32_t *block_tables, const int32_t *context_lens,
+                           float scale, void *out, void *workspace,
+                           size_t workspace_bytes_given, void *stream, const char *fn) {
+    Split sp;
+    pkv_status st = check_attn_desc(desc, fn, &sp);
+    if (st) return st;
+    if (desc->dtype != PKV_F16 && desc->dtype != PKV_BF16)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: q/out must be f16 or bf16", fn);
+    if (desc->head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: only head_dim 128 is built", fn);
+    if ((int64_t)desc->num_blocks * desc->num_kv_heads * pkv::kBlock >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_UNSUPPORTED, "%s: pool too large for 32-bit TMA rows", fn);
+    if (desc->num_seqs == 0) return PKV_OK;
+    if (!q || !k_pool || !v_pool || !k_scale || !v_scale || !block_tables || !context_lens ||
+        !out)
+        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
+    if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
+        !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_tables, 4) ||
+        !aligned(context_lens, 4))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID, "%s: scale is not finite", fn);
+    const size_t need = workspace_bytes(desc, sp);
+    if (need) {
+        if (!workspace || workspace_bytes_given < need)
+            return fail(PKV_ERR_INVALID, "%s: workspace needs %zu bytes", fn, need);
+        if (!aligned(workspace, 256))
+            return fail(PKV_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+    }
+    pkv::DecodeFp8Params fp;
+    pkv::DecodeParams &prm = fp.base;
+    prm.q = q;
+    prm.k_pool = k_pool;
+    prm.v_pool = v_pool;
+    prm.k_new = k_new;
+    prm.v_new = v_new;
+    prm.slot_mapping = slot_mapping;
+    prm.block_tables = block_tables;
+    prm.context_lens = context_lens;
+    prm.out = out;
+    const size_t rows = (size_t)desc->num_seqs * desc->num_q_heads * sp.pmax;
+    prm.ws_o = need ? static_cast<float *>(workspace) : nullptr;
+    prm.ws_ml = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 round_up(rows * desc->head_dim * 4, 256))
+                     : nullptr;
+    prm.S = desc->num_seqs;
+    prm.Hq = desc->num_q_heads;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.maxB = desc->max_blocks_per_seq;
+    prm.part_blocks = sp.part_blocks;
+    prm.pmax = sp.pmax;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    fp.k_scale = k_scale;
+    fp.v_scale = v_scale;
+    const int g = desc->num_q_heads / desc->num_kv_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (desc->dtype == PKV_F16) return dispatch_fp8<__half>(g, fp, s);
+    return dispatch_fp8<__nv_bfloat16>(g, fp, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -529,59 +594,28 @@ pkv_status paged_attn_decode_fp8(const pkv_attn_desc *desc, const void *q, const
                                  const float *v_scale, const int32_t *block_tables,
                                  const int32_t *context_lens, float scale, void *out,
                                  void *workspace, size_t workspace_bytes_given, void *stream) {
-    const char *fn = "paged_attn_decode_fp8";
-    Split sp;
-    pkv_status st = check_attn_desc(desc, fn, &sp);
-    if (st) return st;
-    if (desc->dtype != PKV_F16 && desc->dtype != PKV_BF16)
-        return fail(PKV_ERR_UNSUPPORTED, "%s: q/out must be f16 or bf16", fn);
-    if (desc->head_dim != 128)
-        return fail(PKV_ERR_UNSUPPORTED, "%s: only head_dim 128 is built", fn);
-    if ((int64_t)desc->num_blocks * desc->num_kv_heads * pkv::kBlock >= ((int64_t)1 << 31))
-        return fail(PKV_ERR_UNSUPPORTED, "%s: pool too large for 32-bit TMA rows", fn);
-    if (desc->num_seqs == 0) return PKV_OK;
-    if (!q || !k_pool || !v_pool || !k_scale || !v_scale || !block_tables || !context_lens ||
-        !out)
-        return fail(PKV_ERR_INVALID, "%s: NULL pointer", fn);
-    if (!aligned(q, 16) || !aligned(k_pool, 16) || !aligned(v_pool, 16) || !aligned(out, 16) ||
-        !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_tables, 4) ||
-        !aligned(context_lens, 4))
-        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
-    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID, "%s: scale is not finite", fn);
-    const size_t need = workspace_bytes(desc, sp);
-    if (need) {
-        if (!workspace || workspace_bytes_given < need)
-            return fail(PKV_ERR_INVALID, "%s: workspace needs %zu bytes", fn, need);
-        if (!aligned(workspace, 256))
-            return fail(PKV_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+    return decode_fp8_impl(desc, q, nullptr, nullptr, nullptr, k_pool, v_pool, k_scale, v_scale,
+                           block_tables, context_lens, scale, out, workspace,
+                           workspace_bytes_given, stream, "paged_attn_decode_fp8");
+}
+
+pkv_status kv_write_fp8_and_decode(const pkv_attn_desc *desc, const void *q, const void *k_new,
+                                   const void *v_new, const int64_t *slot_mapping,
+                                   const float *k_scale, const float *v_scale, void *k_pool,
+                                   void *v_pool, const int32_t *block_tables,
+                                   const int32_t *context_lens, float scale, void *out,
+                                   void *workspace, size_t workspace_bytes_given,
+                                   void *stream) {
+    const char *fn = "kv_write_fp8_and_decode";
+    if (desc && desc->num_seqs > 0) {
+        if (!k_new || !v_new || !slot_mapping)
+            return fail(PKV_ERR_INVALID, "%s: NULL tensor pointer", fn);
+        if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8))
+            return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
     }
-    pkv::DecodeFp8Params fp;
-    pkv::DecodeParams &prm = fp.base;
-    prm.q = q;
-    prm.k_pool = k_pool;
-    prm.v_pool = v_pool;
-    prm.block_tables = block_tables;
-    prm.context_lens = context_lens;
-    prm.out = out;
-    const size_t rows = (size_t)desc->num_seqs * desc->num_q_heads * sp.pmax;
-    prm.ws_o = need ? static_cast<float *>(workspace) : nullptr;
-    prm.ws_ml = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                                 round_up(rows * desc->head_dim * 4, 256))
-                     : nullptr;
-    prm.S = desc->num_seqs;
-    prm.Hq = desc->num_q_heads;
-    prm.Hkv = desc->num_kv_heads;
-    prm.NB = desc->num_blocks;
-    prm.maxB = desc->max_blocks_per_seq;
-    prm.part_blocks = sp.part_blocks;
-    prm.pmax = sp.pmax;
-    prm.scale_log2 = scale * 1.4426950408889634f;
-    fp.k_scale = k_scale;
-    fp.v_scale = v_scale;
-    const int g = desc->num_q_heads / desc->num_kv_heads;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (desc->dtype == PKV_F16) return dispatch_fp8<__half>(g, fp, s);
-    return dispatch_fp8<__nv_bfloat16>(g, fp, s);
+    return decode_fp8_impl(desc, q, k_new, v_new, slot_mapping, k_pool, v_pool, k_scale, v_scale,
+                           block_tables, context_lens, scale, out, workspace,
+                           workspace_bytes_given, stream, fn);
 }
 
 }  // extern "C"

@@ -26,6 +26,10 @@ def bits(t):
     return W.to_numpy_bits(t)
 
 
+def u8(t):
+    return t.detach().cpu().contiguous().numpy()
+
+
 def fused_and_separate(wl, vals, slots, pt):
     """Run the fused call on one copy of the pools and kv_write + paged_attn_decode on
     another; return (out_fused, out_separate, pools_fused, pools_separate)."""
@@ -98,9 +102,89 @@ def test_fused_refuses_a_slot_that_is_not_the_newest_position():
     assert torch.isfinite(out).all()
 
 
-def test_fused_full_size_gqa_matches_separate_calls():
-    wl = W.gqa()
+@pytest.mark.parametrize("name", ["opt13b", "gqa", "long"])
+def test_fused_full_size_matches_separate_calls(name):
+    """The bench's default launch configuration at full size: bit-identical to the two
+    separate calls (which the full-size sampled oracle tests cover)."""
+    wl = W.CONFIGS[name]()
     vals = W.make_values(wl, "cuda")
     out1, out2, (kp1, vp1), (kp2, vp2) = fused_and_separate(wl, vals, wl.slot_mapping, 0)
     assert torch.equal(kp1, kp2) and torch.equal(vp1, vp2)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (16, 2)])
+@pytest.mark.parametrize("pt", [0, 64])
+def test_fused_fp8_step_matches_oracle_and_separate_calls(dtype, Hq, Hkv, pt):
+    wl = W.make_workload("f8", RAGGED, Hq, Hkv, 128, dtype, 17 * Hq + Hkv + pt,
+                         pool_factor=1.3, partition_tokens=pt)
+    vals = {k: v.cuda() for k, v in W.make_values_fp8(wl, "cpu").items()}
+    kp2, vp2 = vals["k_pool"].clone(), vals["v_pool"].clone()
+    kp0, vp0 = u8(vals["k_pool"]).copy(), u8(vals["v_pool"]).copy()
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    sl = torch.from_numpy(wl.slot_mapping).cuda()
+    slots = wl.slot_mapping.copy()
+    sl[::4] = -1
+    slots[::4] = -1
+    out1 = B.kv_write_fp8_and_decode(vals["q"], vals["k_new"], vals["v_new"], sl,
+                                     vals["k_scale"], vals["v_scale"], vals["k_pool"],
+                                     vals["v_pool"], bt, lens, wl.scale, partition_tokens=pt)
+    B.kv_write_fp8(vals["k_new"], vals["v_new"], sl, vals["k_scale"], vals["v_scale"], kp2, vp2)
+    out2 = B.paged_attn_decode_fp8(vals["q"], kp2, vp2, vals["k_scale"], vals["v_scale"], bt,
+                                   lens, wl.scale, partition_tokens=pt)
+    torch.cuda.synchronize()
+    assert torch.equal(vals["k_pool"], kp2) and torch.equal(vals["v_pool"], vp2)
+    assert np.array_equal(bits(out1), bits(out2))
+    ks, vs = vals["k_scale"].cpu().numpy(), vals["v_scale"].cpu().numpy()
+    oracle.kv_write_fp8(bits(vals["k_new"]), bits(vals["v_new"]), slots, ks, vs, kp0, vp0, dtype)
+    assert np.array_equal(u8(vals["k_pool"]), kp0) and np.array_equal(u8(vals["v_pool"]), vp0)
+    ref = oracle.paged_attn_decode_fp8(bits(vals["q"]), kp0, vp0, ks, vs, wl.block_tables,
+                                       wl.context_lens, wl.scale, dtype)
+    err = np.max(np.abs(out1.double().cpu().numpy() - ref))
+    assert err <= TOL[dtype], err
+
+
+def test_fused_fp8_refuses_a_slot_that_is_not_the_newest_position():
+    wl = W.make_workload("f8bad", [20, 40, 33], 8, 2, 128, "bf16", 7, pool_factor=1.5)
+    vals = {k: v.cuda() for k, v in W.make_values_fp8(wl, "cpu").items()}
+    kp0, vp0 = vals["k_pool"].clone(), vals["v_pool"].clone()
+    slots = wl.slot_mapping.copy()
+    slots[2] -= 1
+    sl = torch.from_numpy(slots).cuda()
+    B.kv_write_fp8_and_decode(vals["q"], vals["k_new"], vals["v_new"], sl, vals["k_scale"],
+                              vals["v_scale"], vals["k_pool"], vals["v_pool"],
+                              torch.from_numpy(wl.block_tables).cuda(),
+                              torch.from_numpy(wl.context_lens).cuda(), wl.scale)
+    assert B.device_faults() == ["bad slot"]
+    sl_ok = torch.from_numpy(wl.slot_mapping).cuda()
+    sl_ok[2] = -1                     # what should have been written: sequences 0 and 1
+    B.kv_write_fp8(vals["k_new"], vals["v_new"], sl_ok, vals["k_scale"], vals["v_scale"], kp0,
+                   vp0)
+    torch.cuda.synchronize()
+    assert torch.equal(vals["k_pool"], kp0) and torch.equal(vals["v_pool"], vp0)
+
+
+def test_fused_fp8_full_size_gqa_sampled():
+    wl = W.gqa()
+    vals = W.make_values_fp8(wl, "cuda")
+    kp0, vp0 = u8(vals["k_pool"]).copy(), u8(vals["v_pool"]).copy()
+    out = B.kv_write_fp8_and_decode(vals["q"], vals["k_new"], vals["v_new"],
+                                    torch.from_numpy(wl.slot_mapping).cuda(), vals["k_scale"],
+                                    vals["v_scale"], vals["k_pool"], vals["v_pool"],
+                                    torch.from_numpy(wl.block_tables).cuda(),
+                                    torch.from_numpy(wl.context_lens).cuda(), wl.scale)
+    torch.cuda.synchronize()
+    ks, vs = u8(vals["k_scale"]), u8(vals["v_scale"])
+    oracle.kv_write_fp8(bits(vals["k_new"]), bits(vals["v_new"]), wl.slot_mapping, ks, vs, kp0,
+                        vp0, "bf16")
+    assert np.array_equal(u8(vals["k_pool"]), kp0) and np.array_equal(u8(vals["v_pool"]), vp0)
+    rng = np.random.default_rng(3)
+    rows = np.stack([rng.integers(0, wl.num_seqs, 40), rng.integers(0, 32, 40)], 1)
+    rows[0] = (int(np.argmax(wl.context_lens)), 31)
+    rows = rows.astype(np.int32)
+    ref = oracle.paged_attn_decode_fp8(bits(vals["q"]), kp0, vp0, ks, vs, wl.block_tables,
+                                       wl.context_lens, wl.scale, "bf16", rows=rows)
+    got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
+    assert np.max(np.abs(got - ref)) <= TOL["bf16"]
