@@ -40,6 +40,27 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t 
     return t - ((t >> 1) & 0x3F803F80u);
 }
 
+// How many of the 8 P.V m-tiles (16 head dims each) widen V on the conversion unit (XU
+// pipe, exact values); the others use the integer trick above (ALU pipe, values x 2^-8).
+#ifndef PKV_FP8_CVT_TILES
+#define PKV_FP8_CVT_TILES 4
+#endif
+constexpr int kCvtTiles = PKV_FP8_CVT_TILES;
+
+// Two E4M3 codes (low byte first) to an f16x2 register, exactly, on the conversion unit.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// 2^x with the hardware approximation, results below 2^-126 flushed to zero (weights that
+// small vanish next to the largest one, which is at least 1).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // D = A * B + C for one m16n8k32 tile of E4M3 codes, fp32 accumulators.
 __device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {
@@ -351,42 +372,32 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
 
         // ---- online softmax (lane: tokens g, g+8 of heads 2tq, 2tq+1) --------------------
-        const float x0 = g < nvalid ? sacc[0] * sl0 : -INFINITY;
-        const float x1 = g < nvalid ? sacc[1] * sl1 : -INFINITY;
-        const float x2 = g + 8 < nvalid ? sacc[2] * sl0 : -INFINITY;
-        const float x3 = g + 8 < nvalid ? sacc[3] * sl1 : -INFINITY;
-        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
-            bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
+        float x0 = sacc[0] * sl0, x1 = sacc[1] * sl1, x2 = sacc[2] * sl0, x3 = sacc[3] * sl1;
+        if (nvalid < kBlock) {  // the sequence's last block: no weight past its end
+            x0 = g < nvalid ? x0 : -INFINITY;
+            x1 = g < nvalid ? x1 : -INFINITY;
+            x2 = g + 8 < nvalid ? x2 : -INFINITY;
+            x3 = g + 8 < nvalid ? x3 : -INFINITY;
         }
-        // Lazy rescale: the reference max moves only when a block's max passes it by more
-        // than kLazyRescale (base 2), so P stays <= 2^kLazyRescale (f16 holds it) and most
-        // blocks skip the rescale of O; O / l is unchanged by the choice of reference.
-        const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
-        const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
-        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-        const float a0 = mn0 == m_run[0] ? 1.f : exp2f(m_run[0] - mn0);
-        const float a1 = mn1 == m_run[1] ? 1.f : exp2f(m_run[1] - mn1);
-        float s0 = p0 + p2, s1 = p1 + p3;
+        // Lazy rescale: a head's reference max moves only when a block's max passes it by
+        // more than kLazyRescale (base 2), so P stays <= 2^kLazyRescale (f16 holds it); O / l
+        // does not depend on the reference.  One vote tells whether any score passes its
+        // reference by that much; only then (a warp's first block, and rarely after) does
+        // the warp reduce the block's max and rescale O and its partial sums.
+        if (__any_sync(FULL, fmaxf(x0, x2) > m_run[0] + kLazyRescale ||
+                                 fmaxf(x1, x3) > m_run[1] + kLazyRescale)) {
+            float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            s0 += __shfl_xor_sync(FULL, s0, m);
-            s1 += __shfl_xor_sync(FULL, s1, m);
-        }
-        l_run[0] = l_run[0] * a0 + s0;
-        l_run[1] = l_run[1] * a1 + s1;
-        m_run[0] = mn0;
-        m_run[1] = mn1;
-
-        // P^T fragments: b0 holds tokens 2tq, 2tq+1 and b1 tokens 8+2tq, 9+2tq of head g,
-        // which are the slots 4tq..4tq+3 a lane reads from a V^T row.
-        const uint32_t b0 = movmatrix_trans(f32x2_to_f16x2(p0, p1));
-        const uint32_t b1 = movmatrix_trans(f32x2_to_f16x2(p2, p3));
-
-        if (__any_sync(FULL, a0 != 1.f || a1 != 1.f)) {
+            for (int m = 4; m < 32; m <<= 1) {
+                bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
+                bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
+            }
+            const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
+            const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
+            const float a0 = mn0 == m_run[0] ? 1.f : ex2_ftz(m_run[0] - mn0);
+            const float a1 = mn1 == m_run[1] ? 1.f : ex2_ftz(m_run[1] - mn1);
+            l_run[0] *= a0;
+            l_run[1] *= a1;
 #pragma unroll
             for (int t = 0; t < KSTEPS; ++t) {
                 o[t][0] *= a0;
@@ -394,7 +405,19 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                 o[t][2] *= a0;
                 o[t][3] *= a1;
             }
+            m_run[0] = mn0;
+            m_run[1] = mn1;
         }
+        const float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
+        const float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+        // per-lane partial sums; the 8 token-row lanes of a head add theirs after the loop
+        l_run[0] += p0 + p2;
+        l_run[1] += p1 + p3;
+
+        // P^T fragments: b0 holds tokens 2tq, 2tq+1 and b1 tokens 8+2tq, 9+2tq of head g,
+        // which are the slots 4tq..4tq+3 a lane reads from a V^T row.
+        const uint32_t b0 = movmatrix_trans(f32x2_to_f16x2(p0, p1));
+        const uint32_t b1 = movmatrix_trans(f32x2_to_f16x2(p2, p3));
 
         // ---- O^T += V^T P^T -----------------------------------------------------------------
         const uint32_t vb = smem_u32(Vs);
@@ -404,12 +427,19 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             ldmatrix_x4(r, vb + (32 * t2 + v_row) * 16);
             // r[0]: dims 32t2+0..7, r[1]: +8..15 (m-tile 2t2); r[2], r[3]: m-tile 2t2+1
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {  // V x 2^-8 widened to f16 on the integer pipe
+            for (int h = 0; h < 2; ++h) {
                 uint32_t a[4];
-                a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x1404u);
-                a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x3424u);
-                a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x1404u);
-                a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x3424u);
+                if (2 * t2 + h < kCvtTiles) {
+                    a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] & 0xffffu));
+                    a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] >> 16));
+                    a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] & 0xffffu));
+                    a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] >> 16));
+                } else {
+                    a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x1404u);
+                    a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x3424u);
+                    a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x1404u);
+                    a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x3424u);
+                }
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }
         }
@@ -431,13 +461,21 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
     }
 
+#pragma unroll
+    for (int m = 4; m < 32; m <<= 1) {
+        l_run[0] += __shfl_xor_sync(FULL, l_run[0], m);
+        l_run[1] += __shfl_xor_sync(FULL, l_run[1], m);
+    }
+
     __syncthreads();  // every warp is done with its ring: the merge states go over it
-    const float vsc = fp.v_scale[hk] * 256.f;  // the integer widening scaled V by 2^-8
+    // m-tiles widened on the integer pipe carry V x 2^-8
+    const float vsc_cvt = fp.v_scale[hk], vsc_int = vsc_cvt * 256.f;
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
     if (h0 < G) {
         float *dst = mo + (warp * G + h0) * D;
 #pragma unroll
         for (int t = 0; t < KSTEPS; ++t) {
+            const float vsc = t < kCvtTiles ? vsc_cvt : vsc_int;
             dst[16 * t + g] = o[t][0] * vsc;
             dst[16 * t + g + 8] = o[t][2] * vsc;
         }
@@ -450,6 +488,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         float *dst = mo + (warp * G + h1) * D;
 #pragma unroll
         for (int t = 0; t < KSTEPS; ++t) {
+            const float vsc = t < kCvtTiles ? vsc_cvt : vsc_int;
             dst[16 * t + g] = o[t][1] * vsc;
             dst[16 * t + g + 8] = o[t][3] * vsc;
         }
