@@ -53,14 +53,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
-// 2^x with the hardware approximation, results below 2^-126 flushed to zero (weights that
-// small vanish next to the largest one, which is at least 1).
-__device__ __forceinline__ float ex2_ftz(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // D = A * B + C for one m16n8k32 tile of E4M3 codes, fp32 accumulators.
 __device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4],
                                                uint32_t b0, uint32_t b1) {

@@ -212,39 +212,32 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
         }
 
         // ---- online softmax: lane holds tokens g, g+8 of heads 2tq, 2tq+1 ------------
-        const float x0 = g < nvalid ? sacc[0] * sl : -INFINITY;
-        const float x1 = g < nvalid ? sacc[1] * sl : -INFINITY;
-        const float x2 = g + 8 < nvalid ? sacc[2] * sl : -INFINITY;
-        const float x3 = g + 8 < nvalid ? sacc[3] * sl : -INFINITY;
-        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
-            bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
+        float x0 = sacc[0] * sl, x1 = sacc[1] * sl, x2 = sacc[2] * sl, x3 = sacc[3] * sl;
+        if (nvalid < kBlock) {  // the sequence's last block: no weight past its end
+            x0 = g < nvalid ? x0 : -INFINITY;
+            x1 = g < nvalid ? x1 : -INFINITY;
+            x2 = g + 8 < nvalid ? x2 : -INFINITY;
+            x3 = g + 8 < nvalid ? x3 : -INFINITY;
         }
-        // lazy rescale: the reference max moves only past a margin of kLazyRescale
-        const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
-        const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
-        const float p0 = exp2f(x0 - mn0), p1 = exp2f(x1 - mn1);
-        const float p2 = exp2f(x2 - mn0), p3 = exp2f(x3 - mn1);
-        const float a0 = mn0 == m_run[0] ? 1.f : exp2f(m_run[0] - mn0);
-        const float a1 = mn1 == m_run[1] ? 1.f : exp2f(m_run[1] - mn1);
-        float s0 = p0 + p2, s1 = p1 + p3;
+        // Lazy rescale: a head's reference max moves only when a block's max passes it by
+        // more than kLazyRescale (base 2), so P stays <= 2^kLazyRescale; O / l does not
+        // depend on the reference.  One vote tells whether any score passes its reference
+        // by that much; only then (a warp's first block, and rarely after) does the warp
+        // reduce the block's max and rescale O and its partial sums.
+        if (__any_sync(FULL, fmaxf(x0, x2) > m_run[0] + kLazyRescale ||
+                                 fmaxf(x1, x3) > m_run[1] + kLazyRescale)) {
+            float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
 #pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            s0 += __shfl_xor_sync(FULL, s0, m);
-            s1 += __shfl_xor_sync(FULL, s1, m);
-        }
-        l_run[0] = l_run[0] * a0 + s0;
-        l_run[1] = l_run[1] * a1 + s1;
-        m_run[0] = mn0;
-        m_run[1] = mn1;
-
-        // P^T fragments (k = token, n = head) by transposing the two 8x8 halves of P
-        const uint32_t b0 = movmatrix_trans(pack2<BF>(p0, p1));
-        const uint32_t b1 = movmatrix_trans(pack2<BF>(p2, p3));
-
-        if (__any_sync(FULL, a0 != 1.f || a1 != 1.f)) {
+            for (int m = 4; m < 32; m <<= 1) {
+                bm0 = fmaxf(bm0, __shfl_xor_sync(FULL, bm0, m));
+                bm1 = fmaxf(bm1, __shfl_xor_sync(FULL, bm1, m));
+            }
+            const float mn0 = bm0 > m_run[0] + kLazyRescale ? bm0 : m_run[0];
+            const float mn1 = bm1 > m_run[1] + kLazyRescale ? bm1 : m_run[1];
+            const float a0 = mn0 == m_run[0] ? 1.f : ex2_ftz(m_run[0] - mn0);
+            const float a1 = mn1 == m_run[1] ? 1.f : ex2_ftz(m_run[1] - mn1);
+            l_run[0] *= a0;
+            l_run[1] *= a1;
 #pragma unroll
             for (int t = 0; t < KSTEPS; ++t) {
                 o[t][0] *= a0;
@@ -252,7 +245,18 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                 o[t][2] *= a0;
                 o[t][3] *= a1;
             }
+            m_run[0] = mn0;
+            m_run[1] = mn1;
         }
+        const float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
+        const float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+        // per-lane partial sums; the 8 token-row lanes of a head add theirs after the loop
+        l_run[0] += p0 + p2;
+        l_run[1] += p1 + p3;
+
+        // P^T fragments (k = token, n = head) by transposing the two 8x8 halves of P
+        const uint32_t b0 = movmatrix_trans(pack2<BF>(p0, p1));
+        const uint32_t b1 = movmatrix_trans(pack2<BF>(p2, p3));
 
         // ---- O^T += V^T P^T ------------------------------------------------------------
         const uint32_t vb = smem_u32(Vs);
@@ -281,6 +285,12 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
         for (int t = 0; t < KSTEPS; ++t)
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+    }
+
+#pragma unroll
+    for (int m = 4; m < 32; m <<= 1) {
+        l_run[0] += __shfl_xor_sync(FULL, l_run[0], m);
+        l_run[1] += __shfl_xor_sync(FULL, l_run[1], m);
     }
 
     // ---- warp state -> shared memory; heads 2tq and 2tq+1 of this lane ----------------

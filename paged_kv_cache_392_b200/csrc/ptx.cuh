@@ -78,6 +78,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
+// 2^x with the hardware approximation, results below 2^-126 flushed to zero (softmax weights
+// that small vanish next to the largest one, which is at least 1).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // L2 policy: stream through (evict first).  Used for K/V blocks that one CTA reads once.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;
