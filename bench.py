@@ -512,7 +512,9 @@ def run_pkv(args):
     ws_bytes = B.attn_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     npairs = len(pairs)
-    rows_split, pmax = split_rows(wl, pt)
+    # the partition the library will use (the FP8 decode may pick a wider one)
+    pt_run = B.fp8_partition_tokens(desc) if fp8 else (pt or 512)
+    rows_split, pmax = split_rows(wl, pt_run)
     nbytes = algorithmic_bytes(wl, pairs, rows_split, kv_es=1 if fp8 else None)
 
     # The newest token's write runs inside the decode kernel (kv_write_and_decode,
@@ -759,7 +761,7 @@ def run_pkv(args):
                 "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
                 "block_size": 16, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
                 "context_tokens": int(wl.context_lens.sum()),
-                "partition_tokens": pt or 512, "cow_pairs_per_step": npairs,
+                "partition_tokens": pt_run, "cow_pairs_per_step": npairs,
                 "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
                 "l2": "no flush: KV working set %.2f GB per step > 126 MB L2" %
                       (nbytes["kv"] / 1e9),

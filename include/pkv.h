@@ -203,6 +203,15 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  * Scores and the weighted sum run on the codes widened to f16 with fp32 accumulation; the
  * K scale multiplies the scores and the V scale the output.
  */
+/*
+ * Partition size, in tokens, that paged_attn_decode_fp8 / kv_write_fp8_and_decode use for
+ * this descriptor on the current device: desc->partition_tokens when it is set; otherwise
+ * the library's choice, 512, or 2048 when the batch's (sequence, kv head) pairs alone give
+ * at least four CTAs per resident CTA slot.  Never needs more workspace than
+ * pkv_attn_workspace_bytes(desc).  Returns 0 and sets the last error on an invalid desc.
+ */
+int32_t pkv_fp8_partition_tokens(const pkv_attn_desc *desc);
+
 pkv_status kv_write_fp8(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
                         const int64_t *slot_mapping, int32_t num_tokens, const float *k_scale,
                         const float *v_scale, void *k_pool, void *v_pool, void *stream);

@@ -31,7 +31,7 @@ EXPORTS = [
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
     "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
-    "kv_write_and_decode", "kv_write_fp8_and_decode",
+    "kv_write_and_decode", "kv_write_fp8_and_decode", "pkv_fp8_partition_tokens",
 ]
 
 
@@ -70,6 +70,7 @@ def lib():
         "pkv_last_error": ([], ctypes.c_char_p),
         "pkv_version": ([], ctypes.c_char_p),
         "pkv_attn_workspace_bytes": ([dp], sz),
+        "pkv_fp8_partition_tokens": ([dp], i32),
         "paged_attn_decode": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz, vp], i32),
         "paged_attn_decode_no_alloc": ([dp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp], i32),
         "kv_write": ([dp, vp, vp, vp, i32, vp, vp, vp], i32),
@@ -172,6 +173,14 @@ def attn_workspace_bytes(desc):
     err = last_error()
     if n == 0 and err:
         raise PkvError(1, err)
+    return n
+
+
+def fp8_partition_tokens(desc):
+    """Partition size (tokens) the FP8 decode uses for ``desc`` on the current device."""
+    n = lib().pkv_fp8_partition_tokens(ctypes.byref(desc))
+    if n == 0:
+        raise PkvError(1, last_error())
     return n
 
 

@@ -131,3 +131,32 @@ def test_fp8_blocks_copy_and_swap_bit_exact():
     ek[[30, 31]] = kp[[1, 5]]
     ev[[30, 31]] = vp[[1, 5]]
     assert torch.equal(dk.cpu(), ek) and torch.equal(dv.cpu(), ev)
+
+
+def test_decode_fp8_full_size_opt13b_sampled():
+    """The OPT-13B-shaped batch in the bench's launch configuration: one query head per kv
+    head (4 warps per CTA) and the library's wide FP8 partition, through the fused call."""
+    wl = W.opt13b()
+    vals = W.make_values_fp8(wl, "cuda")
+    desc = B.make_desc(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                       wl.num_blocks, wl.max_blocks_per_seq, vals["q"].dtype)
+    assert B.fp8_partition_tokens(desc) == 2048       # one unit per (sequence, kv head)
+    kp0, vp0 = u8(vals["k_pool"]).copy(), u8(vals["v_pool"]).copy()
+    out = B.kv_write_fp8_and_decode(vals["q"], vals["k_new"], vals["v_new"],
+                                    torch.from_numpy(wl.slot_mapping).cuda(), vals["k_scale"],
+                                    vals["v_scale"], vals["k_pool"], vals["v_pool"],
+                                    torch.from_numpy(wl.block_tables).cuda(),
+                                    torch.from_numpy(wl.context_lens).cuda(), wl.scale)
+    torch.cuda.synchronize()
+    ks, vs = u8(vals["k_scale"]), u8(vals["v_scale"])
+    oracle.kv_write_fp8(bits(vals["k_new"]), bits(vals["v_new"]), wl.slot_mapping, ks, vs, kp0,
+                        vp0, "f16")
+    assert np.array_equal(u8(vals["k_pool"]), kp0) and np.array_equal(u8(vals["v_pool"]), vp0)
+    rng = np.random.default_rng(1)
+    rows = np.stack([rng.integers(0, wl.num_seqs, 48), rng.integers(0, 40, 48)], 1)
+    rows[0] = (int(np.argmax(wl.context_lens)), 39)
+    rows = rows.astype(np.int32)
+    ref = oracle.paged_attn_decode_fp8(bits(vals["q"]), kp0, vp0, ks, vs, wl.block_tables,
+                                       wl.context_lens, wl.scale, "f16", rows=rows)
+    got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
+    assert np.max(np.abs(got - ref)) <= TOL["f16"]
