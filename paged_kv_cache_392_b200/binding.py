@@ -25,7 +25,8 @@ BLOCK_SIZE = 16
 # Every symbol include/pkv.h declares.
 EXPORTS = [
     "pkv_last_error", "pkv_version", "pkv_attn_workspace_bytes", "paged_attn_decode",
-    "kv_write", "kv_copy_blocks", "pkv_device_faults", "paged_attn_decode_no_alloc", "pkv_bm_create", "pkv_bm_destroy",
+    "kv_write", "kv_copy_blocks", "pkv_device_faults", "paged_attn_decode_no_alloc",
+    "pkv_bm_create", "pkv_bm_destroy",
     "pkv_bm_add_seq", "pkv_bm_append_slot", "pkv_bm_append_slots", "pkv_bm_fork",
     "pkv_bm_free_seq", "pkv_bm_block_table", "pkv_bm_block_tables", "pkv_bm_seq_len",
     "pkv_bm_refcount", "pkv_bm_num_free", "pkv_bm_num_seqs", "pkv_bm_free_list",

@@ -8,13 +8,14 @@
 //     means code * scale;
 //   * K blocks: [block][kv head][16 tokens][D] bytes (as the 16-bit pools);
 //   * V blocks: [block][kv head][D][16 slots] bytes -- transposed, and slot p of a row holds
-//     token v_slot_token(p) (below), so that a 16-byte row read by one ldmatrix lane quarter
-//     gives the token pairs the P.V tile wants.
+//     token 2*(p>>2) + (p&1) + 8*((p>>1)&1) (v_slot_of_token below is the inverse), so that
+//     the 4 bytes an ldmatrix lane reads from a row are the token pairs the P.V tile wants.
 // Decode: q.K^T runs on m16n8k32 E4M3 tensor-core tiles straight from the K codes, with each
 // query row prescaled by a power of two and split into two E4M3 terms (hi + residual, about
 // bfloat16 precision); P.V widens the V codes exactly to f16 (every E4M3 value is an f16
-// value) for m16n8k16 f16 tiles.  Accumulation is fp32; the K scale (and the q prescale) is
-// folded into the softmax scale and the V scale into the output.  Only D = 128 is built.
+// value; half of the tiles on the integer pipe, half on the conversion unit) for m16n8k16
+// f16 tiles.  Accumulation is fp32; the K scale (and the q prescale) is folded into the
+// softmax scale and the V scale into the output.  Only D = 128 is built.
 #pragma once
 #include <cuda.h>
 #include <cuda_fp8.h>
@@ -146,10 +147,11 @@ struct DecodeFp8Cfg {
     }
 };
 
-// T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.
 // Resident warps per SM the register budget is sized for (16: 128 registers a thread).
 constexpr int kFp8WarpsPerSm = 16;
 
+// T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.  G query heads
+// per kv head, W warps per CTA, NSW ring stages per warp.
 template <typename T, int G, int W, int NSW>
 __global__ void __launch_bounds__(W * 32, kFp8WarpsPerSm / W)
 paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
@@ -247,7 +249,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     float qf_mine = 1.f;
     {
         const bool hv = g < G;
-        const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
+        const T *qrow =
+            static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
         float qv[K32][2][4];
         float amax = 0.f;
 #pragma unroll
@@ -280,12 +283,15 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                 uint32_t hi = 0u, lo = 0u;
 #pragma unroll
                 for (int e = 0; e < 4; e += 2) {
-                    const float2 x = make_float2(qv[j][b][e] * qf_mine, qv[j][b][e + 1] * qf_mine);
-                    const __nv_fp8x2_storage_t h2 = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+                    const float2 x =
+                        make_float2(qv[j][b][e] * qf_mine, qv[j][b][e + 1] * qf_mine);
+                    const __nv_fp8x2_storage_t h2 =
+                        __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
                     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h2, __NV_E4M3);
                     const float2 r = make_float2(x.x - __half2float(__ushort_as_half(hr.x)),
                                                  x.y - __half2float(__ushort_as_half(hr.y)));
-                    const __nv_fp8x2_storage_t l2 = __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
+                    const __nv_fp8x2_storage_t l2 =
+                        __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
                     hi |= static_cast<uint32_t>(h2) << (8 * e);
                     lo |= static_cast<uint32_t>(l2) << (8 * e);
                 }
