@@ -188,3 +188,39 @@ def test_fused_fp8_full_size_gqa_sampled():
                                        wl.context_lens, wl.scale, "bf16", rows=rows)
     got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
     assert np.max(np.abs(got - ref)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("name", ["fork", "beam", "prefix"])
+def test_fused_step_on_sharing_workloads(name):
+    """The bench's step on the block-manager workloads: copy-on-write copies, then the fused
+    write-and-decode; the new tokens land in blocks the copies made private.  Pools bit-exact
+    with the oracle's copy + write, output bit-identical to the separate calls and sampled
+    rows within tolerance of the oracle."""
+    import bench
+    wl, pairs = bench.build_workload(name)
+    d = W.make_values(wl, "cuda")
+    kp0, vp0 = bits(d["k_pool"]).copy(), bits(d["v_pool"]).copy()
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    lens = torch.from_numpy(wl.context_lens).cuda()
+    sl = torch.from_numpy(wl.slot_mapping).cuda()
+    pr = torch.from_numpy(np.ascontiguousarray(pairs, np.int32)).cuda()
+    kp2, vp2 = d["k_pool"].clone(), d["v_pool"].clone()
+    if len(pairs):
+        B.kv_copy_blocks(pr, d["k_pool"], d["v_pool"])
+        B.kv_copy_blocks(pr, kp2, vp2)
+    out = B.kv_write_and_decode(d["q"], d["k_new"], d["v_new"], sl, d["k_pool"], d["v_pool"],
+                                bt, lens, wl.scale)
+    B.kv_write(d["k_new"], d["v_new"], sl, kp2, vp2)
+    out2 = B.paged_attn_decode(d["q"], kp2, vp2, bt, lens, wl.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    oracle.kv_copy_blocks(np.ascontiguousarray(pairs, np.int32), kp0, vp0)
+    oracle.kv_write(bits(d["k_new"]), bits(d["v_new"]), wl.slot_mapping, kp0, vp0)
+    assert np.array_equal(bits(d["k_pool"]), kp0) and np.array_equal(bits(d["v_pool"]), vp0)
+    rng = np.random.default_rng(5)
+    rows = np.stack([rng.integers(0, wl.num_seqs, 24),
+                     rng.integers(0, wl.num_q_heads, 24)], 1).astype(np.int32)
+    ref = oracle.paged_attn_decode(bits(d["q"]), kp0, vp0, wl.block_tables, wl.context_lens,
+                                   wl.scale, wl.dtype, rows=rows)
+    got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
+    assert np.max(np.abs(got - ref)) <= TOL[wl.dtype]
