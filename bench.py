@@ -31,6 +31,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention KV GB/s & seqs/s, % of B200 HBM roofline"
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1000 * 1000     # B200 L2 (126 MB)
 
 WORKLOAD_TEXT = {
     "tiny": "tiny decode step: 4 seqs, context {5,17,33,48}, 2 heads MHA, head_dim 64, fp32, "
@@ -82,6 +83,10 @@ def parse_args(argv=None):
                     help="bracket every E-th decode call of the timed graph with CUDA events "
                          "(the roofline's decode duration); the others run without them, "
                          "since each event node costs about 1 %% of a step")
+    ap.add_argument("--l2-flush", action="store_true",
+                    help="write a 256 MiB buffer before every step, outside the timed work "
+                         "(step and decode calls are then event-bracketed); on by default "
+                         "for workloads whose unique KV bytes fit twice in L2")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
@@ -565,18 +570,31 @@ def run_pkv(args):
     # time.  The decode-call durations come from those events (the last replay's N / E
     # calls).  An event node serialises the stream around it, so bracketing every call
     # would slow the step it measures by about 5 %.
+    # Flush L2 between steps when the bytes a step really reads (shared blocks once) would
+    # fit in it twice over; otherwise the working set itself keeps L2 from carrying over.
+    uniq_kv = (wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim *
+               (1 if fp8 else wl.elem_size) * 2 if "unique_blocks" in wl.extra
+               else nbytes["kv"])
+    flush = args.l2_flush or uniq_kv < 2 * L2_BYTES
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=device) if flush else None
     K = args.steps
     N = max(1, min(50, K))
-    E = max(1, args.decode_events_every)
+    E = 1 if flush else max(1, args.decode_events_every)
     gs = torch.cuda.Stream(device)
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(N)]
     timed = [j for j in range(N) if j % E == 0]
+    # flush mode: an event after the flush of every step marks where the step's own work
+    # starts, so the step time leaves the flush out
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(N)]
 
     def capture(nsteps):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=gs):
             for j in range(nsteps):
+                if scrub is not None:
+                    scrub.fill_(j & 0xFF)       # evict the previous step's lines from L2
+                    evs[j].record(gs)
                 if npairs:
                     B.kv_copy_blocks(pairs_d, kp, vp)
                 write(kn, vn, slots)
@@ -601,13 +619,23 @@ def run_pkv(args):
         t0.record(gs)
         if g_rem is not None:
             g_rem.replay()
-        for _ in range(K // N):
+        # an event after each replay of N steps: the spread of the per-step time
+        rep_ev = [torch.cuda.Event(enable_timing=True) for _ in range(K // N)]
+        for r in range(K // N):
             g_run.replay()
+            rep_ev[r].record(gs)
         t1.record(gs)
         torch.cuda.synchronize()
         barrier(dist, device)
     sampler.stop()
     ms_local = t0.elapsed_time(t1)
+    if scrub is not None:   # step time without the flush: flush end -> decode call end
+        ms_local = statistics.fmean(evs[j].elapsed_time(ev[j][1]) for j in range(N)) * K
+    if scrub is not None:   # the last replay's steps, each without its flush
+        per_step = [evs[j].elapsed_time(ev[j][1]) for j in range(N)]
+    else:                   # one replay of N steps at a time
+        per_step = [rep_ev[r - 1].elapsed_time(rep_ev[r]) / N for r in range(1, len(rep_ev))]
+    step_pcts = (np.percentile(per_step, [10, 50, 90]).tolist() if len(per_step) >= 2 else None)
     ms = max_over_ranks(dist, ms_local, device)
     decode_ms = statistics.fmean(ev[j][0].elapsed_time(ev[j][1]) for j in timed)
     decode_ms = max_over_ranks(dist, decode_ms, device)
@@ -736,7 +764,7 @@ def run_pkv(args):
         # When a step is the decode call alone (fused write, no copy-on-write copies), the
         # step time is that call's duration, taken with no event node inside the loop; the
         # roofline uses it.  Otherwise it uses the event-bracketed calls.
-        only_call = fused and not npairs
+        only_call = fused and not npairs and scrub is None
         bracketed = decode_call_bytes / (decode_ms * 1e-3) / 1e9
         call_ms = step_ms if only_call else decode_ms
         achieved = decode_call_bytes / (call_ms * 1e-3) / 1e9
@@ -751,6 +779,7 @@ def run_pkv(args):
             "steps": K,
             "warmup": args.warmup,
             "ms_per_step": round(step_ms, 5),
+            "ms_per_step_p10_p50_p90": ([round(x, 5) for x in step_pcts] if step_pcts else None),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
@@ -769,8 +798,10 @@ def run_pkv(args):
                 "context_tokens": int(wl.context_lens.sum()),
                 "partition_tokens": pt_run, "cow_pairs_per_step": npairs,
                 "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
-                "l2": "no flush: KV working set %.2f GB per step > 126 MB L2" %
-                      (nbytes["kv"] / 1e9),
+                "l2": ("flushed: 256 MiB written before every step, outside the timed "
+                       "work (step and decode calls event-bracketed)" if scrub is not None
+                       else "no flush: KV working set %.2f GB per step > 126 MB L2" %
+                       (nbytes["kv"] / 1e9)),
                 "parallelism": "replicas x%d" % world,
                 "placement": wl.extra.get("placement", "shuffled"),
                 "kv_write": ("fused into the decode kernel" if fused else
@@ -810,7 +841,9 @@ def run_pkv(args):
                                           "replayed as CUDA graphs)",
                     "serial_value": round(world * nbytes["kv"] / (e2e_serial_ms * 1e-3) / 1e9,
                                           2),
-                    "serial_ms_per_step": round(e2e_serial_ms, 5)},
+                    "serial_ms_per_step": round(e2e_serial_ms, 5),
+                    "l2": "not flushed between steps" if scrub is not None else
+                          "working set larger than L2"},
             "gpu_launches": K * launches_per_step,
             "swap": swap,
             "clocks": sampler.summary(),
