@@ -127,3 +127,18 @@ def test_swap_rejects_host_memory_the_device_cannot_reach(lib):
     assert rc in (1, 4) and B.last_error()
     assert lib.kv_swap_in(ctypes.byref(d), a, -1, a, a, 4, a, a, None) == 1
     assert lib.kv_swap_out(ctypes.byref(d), None, 0, None, None, None, None, 0, None) == 0
+
+
+def test_fp8_partition_choice_reports_the_callers_or_a_library_size(lib):
+    # a partition the caller sets is kept as is
+    assert lib.pkv_fp8_partition_tokens(ctypes.byref(_desc(partition_tokens=256))) == 256
+    # left to the library: 512, or 2048 for batches that fill the GPU on their own (the
+    # wide choice needs a device to count its SMs, so on a host without one it is 512)
+    n = lib.pkv_fp8_partition_tokens(ctypes.byref(_desc()))
+    assert n in (512, 2048)
+    # an invalid descriptor returns 0 and says why
+    assert lib.pkv_fp8_partition_tokens(ctypes.byref(_desc(partition_tokens=24))) == 0
+    assert "multiple of 16" in B.last_error()
+    # the wide choice never needs more scratch than the default split
+    big = _desc(num_seqs=64, num_q_heads=40, num_kv_heads=40, max_blocks_per_seq=128)
+    assert lib.pkv_fp8_partition_tokens(ctypes.byref(big)) in (512, 2048)
