@@ -87,7 +87,7 @@ def parse_args(argv=None):
                     help="write a 256 MiB buffer before every step, outside the timed work "
                          "(step and decode calls are then event-bracketed); on by default "
                          "for workloads whose unique KV bytes fit twice in L2")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args(argv)
 
