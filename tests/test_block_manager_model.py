@@ -194,3 +194,56 @@ def test_swap_fork_cow_traffic_keeps_every_sequence_readable(seed):
         # host blocks are never shared: each belongs to one swapped sequence or is free
         held = [h for s in want if bm.is_swapped(s) for h in bm.block_table(s)]
         assert sorted(held + list(bm.host_free_order())) == list(range(NH))
+
+
+def _planted(name):
+    """A copy of the model class with one plausible mistake in its swap or fork logic."""
+    class Mutant(BlockManagerModel):
+        pass
+
+    if name == "swap_out frees shared blocks":
+        def swap_out(self, seq):
+            table = self.tables[seq]
+            if len(table) > len(self.host_free):
+                raise OutOfBlocks("host pool exhausted")
+            pairs = []
+            for j, blk in enumerate(table):
+                h = self.host_free.popleft()
+                pairs.append((blk, h))
+                if self.ref[blk] > 0:             # drops every holder, not just this one
+                    self.ref[blk] = 0
+                    self.free.append(blk)
+                table[j] = h
+            self.swapped.add(seq)
+            return pairs
+        Mutant.swap_out = swap_out
+    elif name == "swap_in pairs rotated":
+        orig = BlockManagerModel.swap_in
+
+        def swap_in(self, seq):
+            p = orig(self, seq)
+            return [(p[(i + 1) % len(p)][0], g) for i, (_, g) in enumerate(p)]
+        Mutant.swap_in = swap_in
+    elif name == "fork shares without a reference":
+        def fork(self, parent, child):
+            if parent in self.swapped:
+                raise ValueError("parent is swapped out")
+            self.tables[child] = list(self.tables[parent])
+            self.lens[child] = self.lens[parent]     # refcounts not raised
+        Mutant.fork = fork
+    return Mutant
+
+
+@pytest.mark.parametrize("name", ["swap_out frees shared blocks", "swap_in pairs rotated",
+                                  "fork shares without a reference"])
+def test_planted_mistakes_fail_the_data_level_pin(name, monkeypatch):
+    import sys
+    mod = sys.modules[__name__]
+    monkeypatch.setattr(mod, "BlockManagerModel", _planted(name))
+    failed = 0
+    for seed in (0, 1, 2):
+        try:
+            test_swap_fork_cow_traffic_keeps_every_sequence_readable(seed)
+        except (AssertionError, KeyError, ValueError, IndexError, TypeError):
+            failed += 1
+    assert failed > 0, name
