@@ -199,7 +199,9 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  * into the slots of slot_mapping (-1 skips; others range-checked on the device).
  *
  * paged_attn_decode_fp8: as paged_attn_decode, with desc->dtype the type of q and out
- * (PKV_F16 or PKV_BF16); the same workspace rule (pkv_attn_workspace_bytes(desc)).
+ * (PKV_F16 or PKV_BF16); the same workspace rule (pkv_attn_workspace_bytes(desc)).  With
+ * desc->partition_tokens 0 it may split contexts more coarsely than the 16-bit decode;
+ * pkv_fp8_partition_tokens(desc) reports the partition it uses.
  * Scores run on E4M3 tensor-core tiles straight from the K codes (q split into two E4M3
  * terms, about bfloat16 precision); the weighted sum runs on f16 tiles with the V codes
  * widened exactly; accumulation is fp32.  The K scale multiplies the scores and the V scale
