@@ -89,3 +89,30 @@ def test_algorithmic_bytes_and_split_rows():
     rows, pmax = bench.split_rows(wl, 16)
     # lengths 5, 17, 33, 48 over 16-token partitions: 1, 2, 3, 3 partitions
     assert pmax == 3 and rows == (2 + 3 + 3) * 2
+
+
+def test_algorithmic_bytes_of_the_tiny_step_by_hand():
+    """The byte count the roofline divides by, for the tiny workload (4 sequences, lengths
+    5, 17, 33, 48; 2 heads; D 64; fp32), written out term by term."""
+    wl, pairs = bench.build_workload("tiny")
+    nb = bench.algorithmic_bytes(wl, pairs)
+    tokens = 5 + 17 + 33 + 48
+    assert nb["kv"] == tokens * 2 * 64 * 4 * 2                       # K and V, read once
+    qo = 4 * 2 * 64 * 4 * 2                                          # q read, out written
+    tables = (1 + 2 + 3 + 3) * 4 + 4 * 4                             # table entries + lengths
+    assert nb["decode"] == nb["kv"] + qo + tables
+    assert nb["kv_write"] == 4 * 2 * 64 * (4 + 4) * 2 + 4 * 8        # new K/V in, slots out
+    assert nb["kv_copy"] == 0
+    # split: 2 rows x 130 floats written and read per partial state
+    nb2 = bench.algorithmic_bytes(wl, pairs, split_rows=2)
+    assert nb2["decode"] - nb["decode"] == 2 * (64 + 2) * 4 * 2
+    # FP8 pools: one byte per cached K/V element
+    assert bench.algorithmic_bytes(wl, pairs, kv_es=1)["kv"] == tokens * 2 * 64 * 1 * 2
+
+
+def test_split_rows_counts_only_sequences_that_span_partitions():
+    wl, _ = bench.build_workload("tiny")
+    # 16-token partitions: lengths 5 | 17 | 33 | 48 span 1 | 2 | 3 | 3 partitions
+    rows, pmax = bench.split_rows(wl, 16)
+    assert pmax == 3 and rows == (2 + 3 + 3) * wl.num_q_heads
+    assert bench.split_rows(wl, 0) == (0, 1)
