@@ -1,11 +1,15 @@
 """Benchmark of the paged decode path: KV GB/s, sequences/s and fraction of HBM roofline.
 
 One step = one pass of the whole hot path over one batch: copy-on-write block copies (when the
-workload forks), kv_write of each sequence's new token, and paged decode attention (with the
-split / log-sum-exp reduce for sequences longer than one partition).
+workload forks or shares blocks), kv_write of each sequence's new token, and paged decode
+attention (with the split / log-sum-exp reduce for sequences longer than one partition).  By
+default the write runs inside the decode kernel (kv_write_and_decode); --separate-write times
+the two calls.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload opt13b|gqa|long|fork]
-                    [--impl pkv|reference] [--no-cpu-baseline]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload opt13b|gqa|long|fork|beam|prefix|tiny] [--kv-fp8]
+                    [--impl pkv|reference] [--no-cpu-baseline] [--separate-write]
+                    [--l2-flush] [--swap-probe] [--read-probe] [--contiguous]
 
 N > 1 runs under torchrun, one process per GPU; every rank decodes its own replica of the
 batch (weak scaling, no data-path collective); time is the max over ranks.  Rank 0 prints
