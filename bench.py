@@ -93,6 +93,10 @@ def parse_args(argv=None):
                          "for workloads whose unique KV bytes fit twice in L2")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--lib-defines", default="",
+                    help="time a variant build of the library compiled with these macros "
+                         "(space-separated, e.g. '-DPKV_DECODE_FORCE_SIMT' for the "
+                         "CUDA-core decode at every dtype); the line names the variant")
     return ap.parse_args(argv)
 
 
@@ -301,6 +305,56 @@ def split_rows(wl, partition_tokens):
     return int(multi.sum()) * wl.num_q_heads, int(nparts.max())
 
 
+def kv_utilisation(wl):
+    """Fraction of the allocated KV slots that hold a token, from the block tables: every
+    distinct physical block counts 16 slots once, filled as far as the furthest sequence that
+    maps it has written.  Without sharing this is sum(L) / (16 * sum(ceil(L / 16))); the
+    only waste is each sequence's partly filled last block."""
+    fill = {}
+    for s_, L in enumerate(wl.context_lens.astype(np.int64)):
+        nb = -(-int(L) // 16)
+        for j in range(nb):
+            b = int(wl.block_tables[s_, j])
+            fill[b] = max(fill.get(b, 0), min(16, int(L) - 16 * j))
+    slots = 16 * len(fill)
+    return {"tokens_in_blocks": int(sum(fill.values())), "slots_allocated": slots,
+            "frac": round(sum(fill.values()) / slots, 4) if slots else None,
+            "pages_figure": "about 96 % with 16-token blocks (vs 20-38 % for contiguous "
+                            "reservation), OPT-13B on a 40 GB A100"}
+
+
+def uses_l2_flush(args, wl, nbytes, fp8):
+    """Flush L2 between steps when the bytes a step really reads (shared blocks once) would
+    fit in it twice over; otherwise the working set itself keeps L2 from carrying over."""
+    uniq_kv = (wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim *
+               (1 if fp8 else wl.elem_size) * 2 if "unique_blocks" in wl.extra
+               else nbytes["kv"])
+    return bool(args.l2_flush or uniq_kv < 2 * L2_BYTES)
+
+
+def step_config(args, wl, npairs, pt_run, nbytes, flush, fp8):
+    """The line's ``config``: the workload and how a step runs (both arms print the same)."""
+    fused = not args.separate_write
+    return {
+        "workload": WORKLOAD_TEXT[args.workload],
+        "name": args.workload,
+        "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
+        "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+        "block_size": 16, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
+        "context_tokens": int(wl.context_lens.sum()),
+        "partition_tokens": pt_run, "cow_pairs_per_step": npairs,
+        "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
+        "l2": ("flushed: 256 MiB written before every step, outside the timed "
+               "work (step and decode calls event-bracketed)" if flush
+               else "no flush: KV working set %.2f GB per step > 126 MB L2" %
+               (nbytes["kv"] / 1e9)),
+        "parallelism": "replicas x%d" % int(os.environ.get("WORLD_SIZE", "1")),
+        "placement": wl.extra.get("placement", "shuffled"),
+        "kv_write": ("fused into the decode kernel" if fused else
+                     "separate %s kernel" % ("kv_write_fp8" if fp8 else "kv_write")),
+    }
+
+
 # ---- environment: peaks, clocks, profile traffic ----------------------------------------
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -461,6 +515,64 @@ def swap_probe(torch, B, wl, kp, vp, device, reps=5):
     return res
 
 
+def time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ksc, vsc,
+                     nbytes, calls=20, reps=10):
+    """kv_write (or kv_write_fp8) of the step's new tokens and kv_copy_blocks, each timed
+    alone: a CUDA graph of `calls` back-to-back calls replayed `reps` times between CUDA
+    events.  Workloads without copy-on-write pairs copy one block per sequence (its last
+    block into a block no table maps), the most a decode step can need.  Both are small and
+    L2-warm when back to back, so they measure launch-bound kernels as a step runs them."""
+    kv_es = 1 if fp8 else wl.elem_size
+    if len(pairs):
+        cp, source = np.ascontiguousarray(pairs, np.int32), "the step's copy-on-write pairs"
+    else:
+        used = np.zeros(wl.num_blocks, bool)
+        used[wl.block_tables[wl.block_tables >= 0]] = True
+        free = np.flatnonzero(~used)
+        n = min(wl.num_seqs, len(free))
+        last = (wl.context_lens.astype(np.int64) - 1) // 16
+        src = wl.block_tables[np.arange(n), last[:n]]
+        cp = np.stack([src, free[:n]], 1).astype(np.int32)
+        source = "one per sequence: its last block into a block no table maps"
+    cp_d = torch.from_numpy(cp).to(device)
+    copy_bytes = len(cp) * wl.num_kv_heads * 16 * wl.head_dim * kv_es * 2 * 2
+
+    def write():
+        if fp8:
+            B.kv_write_fp8(kn, vn, slots, ksc, vsc, kp, vp)
+        else:
+            B.kv_write(kn, vn, slots, kp, vp)
+
+    res = {}
+    gs = torch.cuda.Stream(device)
+    for name, call, nb in (("kv_write_fp8" if fp8 else "kv_write", write, nbytes["kv_write"]),
+                           ("kv_copy_blocks", lambda: B.kv_copy_blocks(cp_d, kp, vp),
+                            copy_bytes)):
+        with torch.cuda.stream(gs):
+            call()
+        gs.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs):
+            for _ in range(calls):
+                call()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gs):
+            g.replay()
+            a.record(gs)
+            for _ in range(reps):
+                g.replay()
+            b.record(gs)
+        gs.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (calls * reps)
+        res[name] = {"us": round(us, 3), "bytes": int(nb), "gbs": round(nb / (us * 1e-6) / 1e9, 1)}
+        del g
+    res["kv_copy_blocks"]["pairs"] = int(len(cp))
+    res["kv_copy_blocks"]["pairs_source"] = source
+    res["timing"] = ("CUDA graph of %d back-to-back calls replayed %d times, CUDA events; "
+                     "L2-warm" % (calls, reps))
+    return res
+
+
 def read_probe_gbs(torch, device, gib=2, reps=5):
     """Best-of-reps read bandwidth of a plain streaming reduction (torch.sum over a 2 GiB
     bf16 buffer): a read-only ceiling to set beside the copy-based peak."""
@@ -489,12 +601,16 @@ def gpu_uuid(torch, device):
 
 def run_pkv(args):
     import torch
-    from paged_kv_cache_392_b200 import binding as B
     from paged_kv_cache_392_b200 import build as pbuild
+    defines = args.lib_defines.split()
+    if defines:             # before the binding is imported: it loads the library PKV_LIB names
+        os.environ["PKV_LIB"] = pbuild.build(out=pbuild.variant_path(defines), defines=defines)
+    else:
+        pbuild.build()
+    from paged_kv_cache_392_b200 import binding as B
     from paged_kv_cache_392_b200 import workloads as W
 
     world, rank, local = dist_env()
-    pbuild.build()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     dist = init_dist(world)
@@ -574,15 +690,10 @@ def run_pkv(args):
     # time.  The decode-call durations come from those events (the last replay's N / E
     # calls).  An event node serialises the stream around it, so bracketing every call
     # would slow the step it measures by about 5 %.
-    # Flush L2 between steps when the bytes a step really reads (shared blocks once) would
-    # fit in it twice over; otherwise the working set itself keeps L2 from carrying over.
-    uniq_kv = (wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim *
-               (1 if fp8 else wl.elem_size) * 2 if "unique_blocks" in wl.extra
-               else nbytes["kv"])
-    flush = args.l2_flush or uniq_kv < 2 * L2_BYTES
+    flush = uses_l2_flush(args, wl, nbytes, fp8)
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=device) if flush else None
     K = args.steps
-    N = max(1, min(50, K))
+    N = max(1, min(50, K // 4))   # at least 4 replays, so the line carries a spread
     E = 1 if flush else max(1, args.decode_events_every)
     gs = torch.cuda.Stream(device)
     ev = [(torch.cuda.Event(enable_timing=True, external=True),
@@ -759,6 +870,11 @@ def run_pkv(args):
     faults = B.device_faults(clear=True)
     if faults:
         raise RuntimeError("device faults during the end-to-end runs: %s" % faults)
+    aux = time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ksc, vsc,
+                           nbytes)
+    faults = B.device_faults(clear=True)
+    if faults:
+        raise RuntimeError("device faults in the kv_write / kv_copy_blocks timing: %s" % faults)
 
     result = None
     if rank == 0:
@@ -793,24 +909,7 @@ def run_pkv(args):
             "data": "synthetic (seeded), no weights",
             "seqs_per_s": round(world * wl.num_seqs / (step_ms * 1e-3), 1),
             "hbm_frac_step": round(kv_gbs / world / peak, 4),
-            "config": {
-                "workload": WORKLOAD_TEXT[args.workload],
-                "name": args.workload,
-                "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
-                "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-                "block_size": 16, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
-                "context_tokens": int(wl.context_lens.sum()),
-                "partition_tokens": pt_run, "cow_pairs_per_step": npairs,
-                "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
-                "l2": ("flushed: 256 MiB written before every step, outside the timed "
-                       "work (step and decode calls event-bracketed)" if scrub is not None
-                       else "no flush: KV working set %.2f GB per step > 126 MB L2" %
-                       (nbytes["kv"] / 1e9)),
-                "parallelism": "replicas x%d" % world,
-                "placement": wl.extra.get("placement", "shuffled"),
-                "kv_write": ("fused into the decode kernel" if fused else
-                             "separate %s kernel" % ("kv_write_fp8" if fp8 else "kv_write")),
-            },
+            "config": step_config(args, wl, npairs, pt_run, nbytes, scrub is not None, fp8),
             "roofline": {
                 "bound": "hbm",
                 "kernel": "%s (%sdecode + lse_reduce)" % (
@@ -849,6 +948,8 @@ def run_pkv(args):
                     "l2": "not flushed between steps" if scrub is not None else
                           "working set larger than L2"},
             "gpu_launches": K * launches_per_step,
+            "write_and_copy_kernels": aux,
+            "kv_utilisation": kv_utilisation(wl),
             "swap": swap,
             "clocks": sampler.summary(),
         }
@@ -859,6 +960,9 @@ def run_pkv(args):
             result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
         if "sharing" in wl.extra:
             result["sharing"] = wl.extra["sharing"]
+        if defines:
+            result["library"] = {"variant_defines": defines,
+                                 "path": os.path.basename(os.environ["PKV_LIB"])}
         if world == 1 and not args.no_cpu_baseline and not fp8:
             result["cpu_baseline"] = cpu_baseline(wl, vals, args.cpu_seconds)
     if dist is not None:
@@ -888,39 +992,50 @@ def _oracle_rows(wl, seqs):
     return np.array([(s, h) for s in seqs for h in range(wl.num_q_heads)], np.int32)
 
 
-def _calibrate(oracle, wl, host):
+def _calibrate(oracle, wl, host, nthreads=None):
     """Oracle KV bytes per second on this host, from one mid-sized sequence."""
     s = int(np.argsort(wl.context_lens)[wl.num_seqs // 2])
     rows = _oracle_rows(wl, [s])
     t = time.perf_counter()
     oracle.paged_attn_decode(host["q"], host["k_pool"], host["v_pool"], wl.block_tables,
-                             wl.context_lens, wl.scale, wl.dtype, rows=rows)
+                             wl.context_lens, wl.scale, wl.dtype, rows=rows, nthreads=nthreads)
     dt = max(time.perf_counter() - t, 1e-4)
     return _seq_kv_bytes(wl, s) / dt
 
 
-def cpu_baseline(wl, vals, seconds):
-    import oracle
-    from paged_kv_cache_392_b200 import workloads as W
-    host = {k: W.to_numpy_bits(vals[k]) for k in ("q", "k_pool", "v_pool")}
-    rate = _calibrate(oracle, wl, host)
+def _time_oracle(oracle, wl, host, seconds, nthreads=None):
+    """The oracle on a sample of the batch, repeated to about `seconds` of host time."""
+    rate = _calibrate(oracle, wl, host, nthreads)
     seqs, nbytes = _pick_sequences(wl, rate * seconds)
     rows = _oracle_rows(wl, seqs)
     reps, t = 0, time.perf_counter()
     while True:     # repeat the sample (whole batch when it is small) until ~seconds
         oracle.paged_attn_decode(host["q"], host["k_pool"], host["v_pool"], wl.block_tables,
-                                 wl.context_lens, wl.scale, wl.dtype, rows=rows)
+                                 wl.context_lens, wl.scale, wl.dtype, rows=rows,
+                                 nthreads=nthreads)
         reps += 1
         dt = time.perf_counter() - t
         if dt >= 0.8 * seconds or reps >= 1000:
             break
     return {"value": round(reps * nbytes / dt / 1e9, 4), "unit": "GB/s",
-            "cores": oracle.num_threads(), "kind": "oracle",
             "seqs_per_s": round(reps * len(seqs) / dt, 3), "seconds": round(dt, 2),
             "sample": "decode attention of %d of %d sequences (all %d query heads, %d context "
                       "tokens) of the same batch, repeated %d times, fp64, exact two-pass "
                       "softmax" % (len(seqs), wl.num_seqs, wl.num_q_heads,
                                    int(wl.context_lens[seqs].sum()), reps)}
+
+
+def cpu_baseline(wl, vals, seconds):
+    """The oracle on every usable host core (OpenMP over rows), then on one core."""
+    import oracle
+    from paged_kv_cache_392_b200 import workloads as W
+    host = {k: W.to_numpy_bits(vals[k]) for k in ("q", "k_pool", "v_pool")}
+    res = _time_oracle(oracle, wl, host, seconds)
+    res.update({"cores": oracle.num_threads(), "kind": "oracle"})
+    one = _time_oracle(oracle, wl, host, seconds / 3, nthreads=1)
+    one["cores"] = 1
+    res["single_core"] = one
+    return res
 
 
 def run_reference(args):
@@ -931,6 +1046,12 @@ def run_reference(args):
     import torch
     from paged_kv_cache_392_b200 import workloads as W
     wl, pairs = build_workload(args.workload, model_block_manager=True)
+    if args.contiguous:
+        contiguous_placement(wl)
+    pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens
+    pt_run = pt or 512
+    step_bytes = algorithmic_bytes(wl, pairs, split_rows(wl, pt_run)[0])
+    flush = uses_l2_flush(args, wl, step_bytes, False)
     vals = W.make_values(wl, "cpu", torch=torch)
     host = {k: W.to_numpy_bits(v).copy() for k, v in vals.items()}
     rate = _calibrate(oracle, wl, host)
@@ -970,10 +1091,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded), no weights", "impl": "reference",
         "seqs_per_s": round(len(seqs) / dt, 3),
-        "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload,
-                   "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
-                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-                   "block_size": 16, "kv_dtype": wl.dtype},
+        "config": step_config(args, wl, len(pairs), pt_run, step_bytes, flush, False),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "kind": "oracle",
                          "cores": oracle.num_threads(), "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

@@ -11,7 +11,9 @@ import os
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpkv.so")
+# PKV_LIB names another build of the same sources to load instead (a variant compiled with
+# build(out=..., defines=...), such as the CUDA-core-only decode used for A/B measurements).
+LIB_PATH = os.environ.get("PKV_LIB") or os.path.join(HERE, "libpkv.so")
 
 PKV_OK = 0
 STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID", 2: "PKV_ERR_OOM", 3: "PKV_ERR_UNSUPPORTED",
@@ -56,7 +58,8 @@ _lib = None
 
 
 def lib():
-    """Load libpkv.so (built in-tree by ``python -m paged_kv_cache_392_b200.build``)."""
+    """Load libpkv.so (built in-tree by ``python -m paged_kv_cache_392_b200.build``), or the
+    build that ``PKV_LIB`` names."""
     global _lib
     if _lib is not None:
         return _lib

@@ -96,21 +96,18 @@ def test_decode_fp8_ignores_nan_codes_past_the_context():
     assert np.all(np.isfinite(got)) and np.max(np.abs(got - ref)) <= TOL["bf16"]
 
 
-def test_decode_fp8_full_size_gqa_sampled():
+def test_decode_fp8_full_size_gqa_every_row():
     wl = W.gqa()
     v = W.make_values_fp8(wl, "cuda")
     out = B.paged_attn_decode_fp8(v["q"], v["k_pool"], v["v_pool"], v["k_scale"], v["v_scale"],
                                   torch.from_numpy(wl.block_tables).cuda(),
                                   torch.from_numpy(wl.context_lens).cuda(), wl.scale)
-    rng = np.random.default_rng(0)
-    rows = np.stack([rng.integers(0, wl.num_seqs, 40), rng.integers(0, 32, 40)], 1)
-    rows[0] = (int(np.argmax(wl.context_lens)), 31)
-    rows = rows.astype(np.int32)
     ref = oracle.paged_attn_decode_fp8(bits(v["q"]), u8(v["k_pool"]), u8(v["v_pool"]),
                                        u8(v["k_scale"]), u8(v["v_scale"]), wl.block_tables,
-                                       wl.context_lens, wl.scale, "bf16", rows=rows)
-    got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
-    assert np.max(np.abs(got - ref)) <= TOL["bf16"]
+                                       wl.context_lens, wl.scale, "bf16")
+    err = float(np.max(np.abs(out.double().cpu().numpy() - ref)))
+    print("gqa fp8: max abs error over all %d rows: %.3e" % (wl.num_seqs * 32, err))
+    assert err <= TOL["bf16"], err
 
 
 def test_fp8_blocks_copy_and_swap_bit_exact():
@@ -133,7 +130,7 @@ def test_fp8_blocks_copy_and_swap_bit_exact():
     assert torch.equal(dk.cpu(), ek) and torch.equal(dv.cpu(), ev)
 
 
-def test_decode_fp8_full_size_opt13b_sampled():
+def test_decode_fp8_full_size_opt13b_every_row():
     """The OPT-13B-shaped batch in the bench's launch configuration: one query head per kv
     head (4 warps per CTA) and the library's wide FP8 partition, through the fused call."""
     wl = W.opt13b()
@@ -152,11 +149,9 @@ def test_decode_fp8_full_size_opt13b_sampled():
     oracle.kv_write_fp8(bits(vals["k_new"]), bits(vals["v_new"]), wl.slot_mapping, ks, vs, kp0,
                         vp0, "f16")
     assert np.array_equal(u8(vals["k_pool"]), kp0) and np.array_equal(u8(vals["v_pool"]), vp0)
-    rng = np.random.default_rng(1)
-    rows = np.stack([rng.integers(0, wl.num_seqs, 48), rng.integers(0, 40, 48)], 1)
-    rows[0] = (int(np.argmax(wl.context_lens)), 39)
-    rows = rows.astype(np.int32)
     ref = oracle.paged_attn_decode_fp8(bits(vals["q"]), kp0, vp0, ks, vs, wl.block_tables,
-                                       wl.context_lens, wl.scale, "f16", rows=rows)
-    got = out.double().cpu().numpy()[rows[:, 0], rows[:, 1]]
-    assert np.max(np.abs(got - ref)) <= TOL["f16"]
+                                       wl.context_lens, wl.scale, "f16")
+    err = float(np.max(np.abs(out.double().cpu().numpy() - ref)))
+    print("opt13b fp8 (f16 q): max abs error over all %d rows: %.3e (tolerance %g)"
+          % (wl.num_seqs * 40, err, TOL["f16"]))
+    assert err <= TOL["f16"], err
