@@ -57,6 +57,12 @@ typedef enum pkv_dtype { PKV_F32 = 0, PKV_F16 = 1, PKV_BF16 = 2, PKV_FP8_E4M3 = 
                                   /* -1 and not the one of position context_lens[s]-1    */
 #define PKV_FAULT_BAD_PAIR  0x8u  /* copy pair naming a block outside [0, num_blocks)   */
 #define PKV_FAULT_TIMEOUT   0x10u /* a bounded wait on a shared-memory barrier gave up  */
+#define PKV_FAULT_DUPLICATE 0x20u /* kv_write(_fp8): a slot named by two tokens of the   */
+                                  /* call; kv_copy_blocks: a destination named by two    */
+                                  /* pairs, or one that is also a source; kv_swap_*: a   */
+                                  /* destination named by two pairs.  Those entries are  */
+                                  /* skipped, the others carried out                      */
+#define PKV_FAULT_BAD_SCALE 0x40u /* FP8: a K or V scale that is not finite and > 0     */
 
 /* Shape of one decode batch and of the pools it reads. */
 typedef struct pkv_attn_desc {
@@ -118,6 +124,11 @@ pkv_status paged_attn_decode(const pkv_attn_desc *desc, const void *q, const voi
  * bytes copied unchanged.  slot_mapping[t] == -1 skips token t.
  *   k_new/v_new  [num_tokens, H_kv, D] dtype
  *   slot_mapping [num_tokens] int64, distinct values in [0, NB*16) or -1
+ * Checked on the device: a slot outside the pool is skipped (PKV_FAULT_BAD_SLOT); a slot
+ * that two or more tokens of the call name is skipped for all of them
+ * (PKV_FAULT_DUPLICATE), so the pools never depend on which write lands last.  The check
+ * compares every slot with every other, num_tokens^2 comparisons in all: nothing next to
+ * the launch at a decode step's size, and about as long as the copy itself for 16k tokens.
  * Only num_kv_heads, head_dim, block_size, num_blocks and dtype of desc are used.
  */
 pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_new,
@@ -156,7 +167,11 @@ pkv_status kv_write_and_decode(const pkv_attn_desc *desc, const void *q, const v
  * pair i, physical block src_dst_pairs[2i+1] of both pools (every kv head and slot) becomes a
  * byte copy of block src_dst_pairs[2i].
  *   src_dst_pairs [num_pairs][2] int32, device memory; destinations distinct and never a
- *                 source of another pair (otherwise the result is unspecified but in bounds)
+ *                 source of any pair
+ * Checked on the device: a pair naming a block outside the pool is skipped
+ * (PKV_FAULT_BAD_PAIR); a pair whose destination another pair also names, or that some pair
+ * (itself included) reads as its source, is skipped (PKV_FAULT_DUPLICATE).  The remaining
+ * pairs are copied, so the result does not depend on the order in which copies run.
  * Only num_kv_heads, head_dim, block_size, num_blocks and dtype of desc are used.
  */
 pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pairs,
@@ -172,8 +187,9 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
  * [num_pairs][2]:
  *   kv_swap_out: (device block, host block) -- host block := device block, K and V;
  *   kv_swap_in:  (host block, device block) -- device block := host block, K and V.
- * Block ids outside their pool are skipped and set PKV_FAULT_BAD_PAIR.  The copies cross
- * PCIe from the kernel itself (one launch per call, whatever the number of blocks).
+ * Block ids outside their pool are skipped and set PKV_FAULT_BAD_PAIR; pairs whose
+ * destination another pair also names are skipped and set PKV_FAULT_DUPLICATE.  The copies
+ * cross PCIe from the kernel itself (one launch per call, whatever the number of blocks).
  * pkv_bm_swap_out / pkv_bm_swap_in produce the pairs.
  */
 pkv_status kv_swap_out(const pkv_attn_desc *desc, const int32_t *pairs, int32_t num_pairs,
@@ -187,16 +203,19 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  * FP8 (E4M3) KV cache ("Memory Optimization in LLM Serving with PagedAttention", section
  * "Broader Context: vLLM, TGI, and TensorRT-LLM": paged KV caches also kept in INT8/FP8).
  * Format (this library's; the page names none):
- *   - k_scale, v_scale: device fp32 [H_kv]; element x is stored as the E4M3 code of
- *     x / scale (fp32 division, round to nearest even, saturating to +-448) and means
- *     code * scale;
+ *   - k_scale, v_scale: device fp32 [H_kv], each finite and > 0; element x is stored as the
+ *     E4M3 code of x / scale (fp32 division, round to nearest even, saturating to +-448)
+ *     and means code * scale.  A head whose K or V scale is not finite and > 0 sets
+ *     PKV_FAULT_BAD_SCALE: the writes skip that head's values and the decode's output for
+ *     its query heads is unspecified;
  *   - k_pool: [NB][H_kv][16][D] bytes;  v_pool: [NB][H_kv][D][16] bytes, transposed, where
  *     slot p of a row holds token 2*(p>>2) + (p&1) + 8*((p>>1)&1) of the block.
  * Only head_dim 128 is built.  Pools are 16-byte aligned.  kv_copy_blocks and kv_swap_* move
  * these blocks with desc->dtype = PKV_FP8_E4M3.
  *
  * kv_write_fp8: desc->dtype is the type of k_new / v_new ([T][H_kv][D]); codes are written
- * into the slots of slot_mapping (-1 skips; others range-checked on the device).
+ * into the slots of slot_mapping (-1 skips; others range-checked on the device, and slots
+ * named twice skipped, as in kv_write).
  *
  * paged_attn_decode_fp8: as paged_attn_decode, with desc->dtype the type of q and out
  * (PKV_F16 or PKV_BF16); the same workspace rule (pkv_attn_workspace_bytes(desc)).  With
@@ -214,6 +233,9 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  * the library's choice, 512, or 2048 when the batch's (sequence, kv head) pairs alone give
  * at least four CTAs per resident CTA slot.  Never needs more workspace than
  * pkv_attn_workspace_bytes(desc).  Returns 0 and sets the last error on an invalid desc.
+ * The library's choice depends on the current device's SM count, and the partition changes
+ * the rounding order of the result: callers that need the same bits on every GPU model
+ * pass an explicit partition_tokens.
  */
 int32_t pkv_fp8_partition_tokens(const pkv_attn_desc *desc);
 
@@ -254,6 +276,9 @@ pkv_status kv_write_fp8_and_decode(const pkv_attn_desc *desc, const void *q, con
  * until the process exits.  It calls no allocating routine.
  *   - The first call on a device looks up that device's copy of the array (once per
  *     device, with that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset (or anything
+ *     else that destroys the device's primary context) it is stale, and this entry point
+ *     must not be called again in that process.
  *   - A batch whose split scratch (pkv_attn_workspace_bytes) exceeds
  *     PKV_STATIC_WORKSPACE_BYTES is rejected with PKV_ERR_INVALID; nothing is launched.
  *   - Every call on a device shares the one array and it keeps the last call's contents

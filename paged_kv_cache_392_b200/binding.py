@@ -19,7 +19,8 @@ PKV_OK = 0
 STATUS = {0: "PKV_OK", 1: "PKV_ERR_INVALID", 2: "PKV_ERR_OOM", 3: "PKV_ERR_UNSUPPORTED",
           4: "PKV_ERR_CUDA", 5: "PKV_ERR_NOT_FOUND"}
 FAULT_BITS = {0x1: "bad context length", 0x2: "bad block id", 0x4: "bad slot",
-              0x8: "bad copy pair", 0x10: "barrier wait timed out"}
+              0x8: "bad copy pair", 0x10: "barrier wait timed out",
+              0x20: "duplicate slot or copy destination", 0x40: "bad fp8 scale"}
 DTYPE_CODE = {torch.float32: 0, torch.float16: 1, torch.bfloat16: 2, torch.uint8: 3}
 PKV_FP8_E4M3 = 3
 BLOCK_SIZE = 16

@@ -48,7 +48,25 @@ constexpr int kBlock = 16;                       // tokens per KV block
 #define PKV_LAZY_RESCALE 8
 #endif
 constexpr float kLazyRescale = float(PKV_LAZY_RESCALE);
-constexpr uint64_t kWaitTimeoutNs = 1000000000;  // bounded shared-memory barrier waits (1 s)
+// Bounded shared-memory barrier waits give up after this long (1 s; test builds shorten it).
+#ifndef PKV_WAIT_TIMEOUT_NS
+#define PKV_WAIT_TIMEOUT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitTimeoutNs = PKV_WAIT_TIMEOUT_NS;
+
+// Test builds only (-DPKV_TEST_WITHHOLD_BLOCK=i): warp 0 of the grid's first CTA issues
+// neither the copy nor the arrival of its i-th block, so its bounded wait on that stage runs
+// out and the timeout path runs (fault bit, drain of the copies still in flight, an empty
+// state for the warp).  No copy targets the withheld stage, so nothing is left in flight.
+__device__ __forceinline__ bool withheld_for_test(int i, int warp) {
+#ifdef PKV_TEST_WITHHOLD_BLOCK
+    return blockIdx.x == 0 && warp == 0 && i == PKV_TEST_WITHHOLD_BLOCK;
+#else
+    (void)i;
+    (void)warp;
+    return false;
+#endif
+}
 
 
 struct DecodeParams {
@@ -98,7 +116,8 @@ __device__ __forceinline__ void write_newest_token(const DecodeParams &p, int s,
             }
             fence_proxy_async_global();
         } else if (lane == 0) {
-            atomicOr(&g_faults, (unsigned)blk < (unsigned)p.NB ? 0x4u : 0x2u);
+            atomicOr(&g_faults,
+                     (unsigned)blk < (unsigned)p.NB ? kFaultBadSlot : kFaultBadBlock);
         }
     }
     __syncwarp();
@@ -275,7 +294,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
 
     const int L = p.context_lens[s];
     if (L < 1 || L > p.maxB * kBlock) {
-        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, 0x1u);
+        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
     const int nblk = (L + kBlock - 1) / kBlock;
@@ -323,7 +342,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
             tab = li < nbw ? btrow[(size_t)W * li] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
-        if (lane == 0) {
+        if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * 2 * CHUNK;
             if ((unsigned)phys < (unsigned)p.NB) {
@@ -333,7 +352,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
                 bulk_g2s(dst, kbase + off, CHUNK, bar, policy);
                 bulk_g2s(dst + CHUNK, vbase + off, CHUNK, bar, policy);
             } else {
-                atomicOr(&g_faults, 0x2u);
+                atomicOr(&g_faults, kFaultBadBlock);
                 mbar_arrive(bar);  // complete the phase without data
             }
         }
@@ -371,7 +390,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
     for (; i < nbw; ++i) {
         const int st = i % NSW;
         if (!mbar_wait_bounded(&bars[st], (uint32_t)(i / NSW) & 1u, kWaitTimeoutNs)) {
-            if (lane == 0) atomicOr(&g_faults, 0x10u);
+            if (lane == 0) atomicOr(&g_faults, kFaultTimeout);
             dead = true;
             break;
         }

@@ -23,6 +23,7 @@
 #include <type_traits>
 
 #include "attn_decode_tc.cuh"
+#include "kv_ops.cuh"
 
 namespace pkv {
 
@@ -85,6 +86,9 @@ __device__ __forceinline__ float load_elem(const void *base, int64_t i) {
         return __bfloat162float(static_cast<const __nv_bfloat16 *>(base)[i]);
 }
 
+// Whether an FP8 scale can encode: finite and above zero (NaN fails both tests).
+__device__ __forceinline__ bool scale_ok(float x) { return x > 0.f && x < INFINITY; }
+
 // E4M3 codes of src[i] / scale and src[i+1] / scale (fp32 division, round to nearest even,
 // saturating to +-448), element i in the low byte: the cache format's quantisation.
 template <typename T>
@@ -98,7 +102,8 @@ __device__ __forceinline__ __nv_fp8x2_storage_t quantize2(const void *src, int64
 // copy the block holding position L-1: quantise the K row and the V column into their slot,
 // then fence the generic-proxy stores against the warp's own TMA / bulk copies of the block.
 // A slot of -1 is skipped; any slot other than position L-1's sets fault bit 4 (bad slot)
-// and is not written.
+// and is not written, and neither is anything when the head's K or V scale is not finite
+// and > 0 (fault bit 0x40).
 template <typename T>
 __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp, int s, int hk,
                                                        int L, int lane) {
@@ -108,7 +113,10 @@ __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp
     if (slot != -1) {
         const int32_t blk = p.block_tables[(size_t)s * p.maxB + (L - 1) / kBlock];
         const int off = (L - 1) % kBlock;
-        if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
+        const float ksc = fp.k_scale[hk], vsc = fp.v_scale[hk];
+        if (!scale_ok(ksc) || !scale_ok(vsc)) {
+            if (lane == 0) atomicOr(&g_faults, kFaultBadScale);
+        } else if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
             const int64_t src = ((int64_t)s * p.Hkv + hk) * D;
             const int64_t hb = (int64_t)blk * p.Hkv + hk;
             const int vs = v_slot_of_token(off);
@@ -116,15 +124,16 @@ __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp
             uint8_t *kp = static_cast<uint8_t *>(const_cast<void *>(p.k_pool));
             uint8_t *vp = static_cast<uint8_t *>(const_cast<void *>(p.v_pool));
             for (int d = 2 * lane; d < D; d += 64) {
-                const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src + d, fp.k_scale[hk]);
-                const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src + d, fp.v_scale[hk]);
+                const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src + d, ksc);
+                const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src + d, vsc);
                 *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + (hb * kBlock + off) * D + d) = kc;
                 vp[(hb * D + d) * kBlock + vs] = static_cast<uint8_t>(vc & 0xffu);
                 vp[(hb * D + d + 1) * kBlock + vs] = static_cast<uint8_t>(vc >> 8);
             }
             fence_proxy_async_global();
         } else if (lane == 0) {
-            atomicOr(&g_faults, (unsigned)blk < (unsigned)p.NB ? 0x4u : 0x2u);
+            atomicOr(&g_faults,
+                     (unsigned)blk < (unsigned)p.NB ? kFaultBadSlot : kFaultBadBlock);
         }
     }
     __syncwarp();
@@ -175,7 +184,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
 
     const int L = p.context_lens[s];
     if (L < 1 || L > p.maxB * kBlock) {
-        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, 0x1u);
+        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
     const int nblk = (L + kBlock - 1) / kBlock;
@@ -218,7 +227,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             tab = li < nbw ? btrow[(size_t)W * li] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
-        if (lane == 0) {
+        if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
             if ((unsigned)phys < (unsigned)p.NB) {
@@ -229,7 +238,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                 bulk_g2s(dst + CHUNK, vbase + (size_t)(phys * p.Hkv + hk) * CHUNK, CHUNK, bar,
                          policy);
             } else {
-                atomicOr(&g_faults, 0x2u);
+                atomicOr(&g_faults, kFaultBadBlock);
                 mbar_arrive(bar);
             }
         }
@@ -307,6 +316,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
     // score scales of this lane's heads 2tq, 2tq+1: softmax scale * K scale / q prescale
+    if (threadIdx.x == 0 && (!scale_ok(fp.k_scale[hk]) || !scale_ok(fp.v_scale[hk])))
+        atomicOr(&g_faults, kFaultBadScale);  // the output of this unit is then unspecified
     const float slk = p.scale_log2 * fp.k_scale[hk];
     const float sl0 = slk / __shfl_sync(FULL, qf_mine, (2 * tq) * 4);
     const float sl1 = slk / __shfl_sync(FULL, qf_mine, (2 * tq + 1) * 4);
@@ -323,7 +334,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     for (; i < nbw; ++i) {
         const int st = i % NSW;
         if (!mbar_wait_bounded(&bars[st], (uint32_t)(i / NSW) & 1u, kWaitTimeoutNs)) {
-            if (lane == 0) atomicOr(&g_faults, 0x10u);
+            if (lane == 0) atomicOr(&g_faults, kFaultTimeout);
             dead = true;
             break;
         }
@@ -512,32 +523,49 @@ struct KvWriteFp8Params {
 };
 
 
-// One thread per (token, head, pair of dims): codes of x / scale, RNE, saturating.
+// grid.x = tile of kTileTokens tokens, grid.y = slice of the tile's (token, head, pair of
+// dims) items, one thread per item: codes of x / scale, RNE, saturating.  Slots shared by
+// two tokens of the call are skipped (PKV_FAULT_DUPLICATE), as in kv_write; a head whose K
+// or V scale is not finite and > 0 is not written (PKV_FAULT_BAD_SCALE).
 template <typename T>
-__global__ void __launch_bounds__(256) kv_write_fp8_kernel(const KvWriteFp8Params p) {
-    const int64_t pairs = (int64_t)p.T * p.Hkv * (p.D / 2);
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= pairs) return;
-    const int d = 2 * (int)(idx % (p.D / 2));
-    const int64_t th = idx / (p.D / 2);
-    const int h = (int)(th % p.Hkv);
-    const int64_t t = th / p.Hkv;
-    const int64_t slot = p.slot_mapping[t];
-    if (slot == -1) return;
-    if (slot < 0 || slot >= (int64_t)p.NB * 16) {
-        if (h == 0 && d == 0) atomicOr(&g_faults, 0x4u);
-        return;
+__global__ void __launch_bounds__(kWriteThreads) kv_write_fp8_kernel(const KvWriteFp8Params p) {
+    __shared__ TileSlots ts;
+    const int64_t t0 = (int64_t)blockIdx.x * kTileTokens;
+    tile_duplicate_slots(p.slot_mapping, p.T, t0, ts);
+    const int ntok = (int)(p.T - t0 < kTileTokens ? p.T - t0 : kTileTokens);
+    const int per_tok = p.Hkv * (p.D / 2);
+    const int items = ntok * per_tok;
+    const int per_cta = (items + gridDim.y - 1) / gridDim.y;
+    const int end = min(items, (int)(blockIdx.y + 1) * per_cta);
+    for (int i = blockIdx.y * per_cta + threadIdx.x; i < end; i += kWriteThreads) {
+        const int tl = i / per_tok, hd = i % per_tok;
+        const int h = hd / (p.D / 2), d = 2 * (hd % (p.D / 2));
+        const int64_t slot = ts.slot[tl];
+        if (slot == -1) continue;
+        if (slot < 0 || slot >= (int64_t)p.NB * 16) {
+            if (hd == 0) atomicOr(&g_faults, kFaultBadSlot);
+            continue;
+        }
+        if ((ts.dup_mask >> tl) & 1u) {
+            if (hd == 0) atomicOr(&g_faults, kFaultDuplicate);
+            continue;
+        }
+        const float ksc = p.k_scale[h], vsc = p.v_scale[h];
+        if (!scale_ok(ksc) || !scale_ok(vsc)) {
+            if (d == 0) atomicOr(&g_faults, kFaultBadScale);
+            continue;
+        }
+        const int64_t blk = slot >> 4;
+        const int off = (int)(slot & 15);
+        const int64_t src = ((t0 + tl) * p.Hkv + h) * p.D + d;
+        const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src, ksc);
+        const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src, vsc);
+        const int64_t hb = blk * p.Hkv + h;
+        *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + (hb * 16 + off) * p.D + d) = kc;
+        const int sp = v_slot_of_token(off);
+        p.v_pool[(hb * p.D + d) * 16 + sp] = static_cast<uint8_t>(vc & 0xffu);
+        p.v_pool[(hb * p.D + d + 1) * 16 + sp] = static_cast<uint8_t>(vc >> 8);
     }
-    const int64_t blk = slot >> 4;
-    const int off = (int)(slot & 15);
-    const int64_t src = th * p.D + d;
-    const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src, p.k_scale[h]);
-    const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src, p.v_scale[h]);
-    const int64_t hb = blk * p.Hkv + h;
-    *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + (hb * 16 + off) * p.D + d) = kc;
-    const int sp = v_slot_of_token(off);
-    p.v_pool[(hb * p.D + d) * 16 + sp] = static_cast<uint8_t>(vc & 0xffu);
-    p.v_pool[(hb * p.D + d + 1) * 16 + sp] = static_cast<uint8_t>(vc >> 8);
 }
 
 }  // namespace pkv

@@ -74,7 +74,7 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
 
     const int L = p.context_lens[s];
     if (L < 1 || L > p.maxB * kBlock) {
-        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, 0x1u);
+        if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
     const int nblk = (L + kBlock - 1) / kBlock;
@@ -120,7 +120,7 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
             tab = li < nbw ? btrow[(size_t)W * li] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
-        if (lane == 0) {
+        if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
             if ((unsigned)phys < (unsigned)p.NB) {
@@ -133,7 +133,7 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
                     tma_load_2d(dst + CHUNK + h * BOX, &tmv, h * 64, row, bar, policy);
                 }
             } else {
-                atomicOr(&g_faults, 0x2u);
+                atomicOr(&g_faults, kFaultBadBlock);
                 mbar_arrive(bar);
             }
         }
@@ -176,7 +176,7 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
     for (; i < nbw; ++i) {
         const int st = i % NSW;
         if (!mbar_wait_bounded(&bars[st], (uint32_t)(i / NSW) & 1u, kWaitTimeoutNs)) {
-            if (lane == 0) atomicOr(&g_faults, 0x10u);
+            if (lane == 0) atomicOr(&g_faults, kFaultTimeout);
             dead = true;
             break;
         }

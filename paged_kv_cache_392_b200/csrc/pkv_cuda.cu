@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cmath>
@@ -244,6 +245,26 @@ pkv_status dispatch_dim(int D, int g, const pkv::DecodeParams &prm, cudaStream_t
     return dispatch_group<T, 128>(g, prm, stream);
 }
 
+int device_sm_count();
+
+// Grid of a kv_write / kv_write_fp8 launch: one row of CTAs per tile of kTileTokens tokens
+// (each CTA checks its tile's slots against the whole call), and as many slices of a tile's
+// `items_per_token * tokens` items as keep about four CTAs per SM busy when there are few
+// tiles (a decode step's write), down to one per tile for long writes, where every slice
+// would repeat the tile's duplicate check.
+pkv_status write_grid(int32_t tokens, int64_t items_per_token, dim3 *grid, const char *fn) {
+    const int64_t tiles = (tokens + pkv::kTileTokens - 1) / pkv::kTileTokens;
+    const int64_t tile_items = items_per_token * std::min<int64_t>(tokens, pkv::kTileTokens);
+    if (tiles > INT_MAX || tile_items > INT_MAX / 2)
+        return fail(PKV_ERR_INVALID, "%s: too many tokens or heads for one launch", fn);
+    const int64_t sms = std::max(1, device_sm_count());
+    const int64_t by_items = (tile_items + pkv::kWriteThreads - 1) / pkv::kWriteThreads;
+    const int64_t by_sms = (4 * sms + tiles - 1) / tiles;
+    const int64_t slices = std::max<int64_t>(1, std::min<int64_t>({by_items, by_sms, 65535}));
+    *grid = dim3((unsigned)tiles, (unsigned)slices);
+    return PKV_OK;
+}
+
 // Shared body of paged_attn_decode and kv_write_and_decode (k_new / v_new / slot_mapping
 // NULL: no fused write).
 pkv_status decode_impl(const pkv_attn_desc *desc, const void *q, const void *k_new,
@@ -373,10 +394,10 @@ pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_
     prm.Hkv = desc->num_kv_heads;
     prm.NB = desc->num_blocks;
     prm.vpr = desc->head_dim * elem_size(desc->dtype) / 16;
-    const int64_t total = 2LL * num_tokens * prm.Hkv * prm.vpr;
-    const int64_t blocks = (total + 255) / 256;
-    if (blocks > INT_MAX) return fail(PKV_ERR_INVALID, "%s: too many tokens", fn);
-    pkv::kv_write_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+    dim3 grid;
+    st = write_grid(num_tokens, 2LL * prm.Hkv * prm.vpr, &grid, fn);
+    if (st) return st;
+    pkv::kv_write_kernel<<<grid, pkv::kWriteThreads, 0, static_cast<cudaStream_t>(stream)>>>(prm);
     return cuda_check(cudaGetLastError(), fn, "launch");
 }
 
@@ -617,16 +638,15 @@ pkv_status kv_write_fp8(const pkv_attn_desc *desc, const void *k_new, const void
     prm.Hkv = desc->num_kv_heads;
     prm.NB = desc->num_blocks;
     prm.D = desc->head_dim;
-    const int64_t total = (int64_t)num_tokens * prm.Hkv * (prm.D / 2);
-    const int64_t blocks = (total + 255) / 256;
-    if (blocks > INT_MAX) return fail(PKV_ERR_INVALID, "%s: too many tokens", fn);
+    dim3 grid;
+    st = write_grid(num_tokens, (int64_t)prm.Hkv * (prm.D / 2), &grid, fn);
+    if (st) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    constexpr int kT = pkv::kWriteThreads;
     switch (desc->dtype) {
-    case PKV_F32: pkv::kv_write_fp8_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(prm); break;
-    case PKV_F16: pkv::kv_write_fp8_kernel<__half><<<(unsigned)blocks, 256, 0, s>>>(prm); break;
-    default:
-        pkv::kv_write_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(prm);
-        break;
+    case PKV_F32: pkv::kv_write_fp8_kernel<float><<<grid, kT, 0, s>>>(prm); break;
+    case PKV_F16: pkv::kv_write_fp8_kernel<__half><<<grid, kT, 0, s>>>(prm); break;
+    default: pkv::kv_write_fp8_kernel<__nv_bfloat16><<<grid, kT, 0, s>>>(prm); break;
     }
     return cuda_check(cudaGetLastError(), fn, "launch");
 }

@@ -142,3 +142,15 @@ def test_fp8_partition_choice_reports_the_callers_or_a_library_size(lib):
     # the wide choice never needs more scratch than the default split
     big = _desc(num_seqs=64, num_q_heads=40, num_kv_heads=40, max_blocks_per_seq=128)
     assert lib.pkv_fp8_partition_tokens(ctypes.byref(big)) in (512, 2048)
+
+
+def test_fault_bits_agree_across_header_binding_and_kernels():
+    """pkv.h's PKV_FAULT_* values, the binding's decoder and the kernels' constants name the
+    same bits."""
+    text = open(HEADER).read()
+    header = {int(v, 16) for v in re.findall(r"#define PKV_FAULT_\w+\s+(0x[0-9a-fA-F]+)u", text)}
+    cuh = open(os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc", "faults.cuh")).read()
+    kernels = {int(v, 16) for v in re.findall(r"constexpr unsigned kFault\w+ = (0x[0-9a-f]+)u",
+                                                cuh)}
+    assert header == kernels == set(B.FAULT_BITS)
+    assert len(header) == 7
