@@ -10,6 +10,7 @@ the two calls.
                     [--workload opt13b|gqa|long|fork|beam|prefix|tiny] [--kv-fp8]
                     [--impl pkv|reference] [--no-cpu-baseline] [--separate-write]
                     [--l2-flush] [--swap-probe] [--read-probe] [--contiguous]
+                    [--layout paged|contiguous] [--decode-only] [--lib-defines '-D...']
 
 N > 1 runs under torchrun, one process per GPU; every rank decodes its own replica of the
 batch (weak scaling, no data-path collective); time is the max over ranks.  Rank 0 prints
@@ -80,6 +81,12 @@ def parse_args(argv=None):
     ap.add_argument("--contiguous", action="store_true",
                     help="place each sequence's blocks contiguously and in order (paged "
                          "kernel over a contiguous layout) instead of shuffled")
+    ap.add_argument("--layout", default="paged", choices=["paged", "contiguous"],
+                    help="contiguous: time attn_decode_contiguous over a [S][H_kv][Lmax][D] "
+                         "cache with no block table (the same tokens, gathered from the "
+                         "pools), decode only; compare with --decode-only on the paged pools")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="the step is the decode call alone (no kv_write)")
     ap.add_argument("--separate-write", action="store_true",
                     help="the newest token's write as its own kernel (kv_write / "
                          "kv_write_fp8) before the decode, instead of the fused call")
@@ -334,8 +341,9 @@ def uses_l2_flush(args, wl, nbytes, fp8):
 
 def step_config(args, wl, npairs, pt_run, nbytes, flush, fp8):
     """The line's ``config``: the workload and how a step runs (both arms print the same)."""
-    fused = not args.separate_write
-    return {
+    decode_only = args.decode_only or args.layout == "contiguous"
+    fused = not args.separate_write and not decode_only
+    cfg = {
         "workload": WORKLOAD_TEXT[args.workload],
         "name": args.workload,
         "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
@@ -350,9 +358,14 @@ def step_config(args, wl, npairs, pt_run, nbytes, flush, fp8):
                (nbytes["kv"] / 1e9)),
         "parallelism": "replicas x%d" % int(os.environ.get("WORLD_SIZE", "1")),
         "placement": wl.extra.get("placement", "shuffled"),
-        "kv_write": ("fused into the decode kernel" if fused else
+        "kv_write": ("none: the step is the decode call alone" if decode_only else
+                     "fused into the decode kernel" if fused else
                      "separate %s kernel" % ("kv_write_fp8" if fp8 else "kv_write")),
     }
+    if args.layout == "contiguous":
+        cfg["layout"] = ("contiguous [S][H_kv][Lmax][D] cache, Lmax = %d, no block table"
+                         % (wl.max_blocks_per_seq * 16))
+    return cfg
 
 
 # ---- environment: peaks, clocks, profile traffic ----------------------------------------
@@ -643,11 +656,30 @@ def run_pkv(args):
     nbytes = algorithmic_bytes(wl, pairs, rows_split, kv_es=1 if fp8 else None)
 
     # The newest token's write runs inside the decode kernel (kv_write_and_decode,
-    # kv_write_fp8_and_decode) unless --separate-write asks for the two calls.
-    fused = not args.separate_write
+    # kv_write_fp8_and_decode) unless --separate-write asks for the two calls, or the step is
+    # the decode alone (--decode-only, --layout contiguous).
+    contig = args.layout == "contiguous"
+    decode_only = args.decode_only or contig
+    if contig and (fp8 or npairs or args.workload in ("fork", "beam", "prefix", "tiny")):
+        raise SystemExit("--layout contiguous applies to the opt13b, gqa and long workloads")
+    fused = not args.separate_write and not decode_only
+    kc = vc = None
+    if contig:      # the same tokens in a [S][H_kv][Lmax][D] reservation per sequence
+        lmax = wl.max_blocks_per_seq * 16
+        kc = torch.zeros((wl.num_seqs, wl.num_kv_heads, lmax, wl.head_dim), dtype=kp.dtype,
+                         device=device)
+        vc = torch.zeros_like(kc)
+        for s_ in range(wl.num_seqs):
+            L = int(wl.context_lens[s_])
+            t = torch.arange(L, device=device)
+            blk = bt[s_].long()[t // 16]
+            kc[s_, :, :L] = kp[blk, :, t % 16].permute(1, 0, 2)
+            vc[s_, :, :L] = vp[blk, :, t % 16].permute(1, 0, 2)
+        nbytes["decode"] -= int(((wl.context_lens + 15) // 16).sum()) * 4 + wl.num_seqs * 4
+        nbytes["step"] = nbytes["decode"]
 
     def write(kn_, vn_, slots_):
-        if fused:
+        if fused or decode_only:
             return
         if fp8:
             B.kv_write_fp8(kn_, vn_, slots_, ksc, vsc, kp, vp)
@@ -655,7 +687,10 @@ def run_pkv(args):
             B.kv_write(kn_, vn_, slots_, kp, vp)
 
     def decode(q_, kn_, vn_, slots_, bt_, lens_, out_):
-        if fp8 and fused:
+        if contig:
+            B.attn_decode_contiguous(q_, kc, vc, lens_, wl.scale, out=out_, workspace=ws,
+                                     partition_tokens=pt)
+        elif fp8 and fused:
             B.kv_write_fp8_and_decode(q_, kn_, vn_, slots_, ksc, vsc, kp, vp, bt_, lens_,
                                       wl.scale, out=out_, workspace=ws, partition_tokens=pt)
         elif fp8:
@@ -674,7 +709,8 @@ def run_pkv(args):
         write(kn, vn, slots)
         decode(q, kn, vn, slots, bt, lens, out)
 
-    launches_per_step = (1 if npairs else 0) + (0 if fused else 1) + 1 + (1 if pmax > 1 else 0)
+    launches_per_step = ((1 if npairs else 0) + (0 if fused or decode_only else 1) + 1 +
+                         (1 if pmax > 1 else 0))
     decode_call_bytes = nbytes["decode"] + (nbytes["kv_write"] if fused else 0)
 
     for _ in range(args.warmup):
@@ -884,11 +920,12 @@ def run_pkv(args):
         # When a step is the decode call alone (fused write, no copy-on-write copies), the
         # step time is that call's duration, taken with no event node inside the loop; the
         # roofline uses it.  Otherwise it uses the event-bracketed calls.
-        only_call = fused and not npairs and scrub is None
+        only_call = (fused or decode_only) and not npairs and scrub is None
         bracketed = decode_call_bytes / (decode_ms * 1e-3) / 1e9
         call_ms = step_ms if only_call else decode_ms
         achieved = decode_call_bytes / (call_ms * 1e-3) / 1e9
-        traffic = None if args.separate_write else profile_traffic(args.workload, fp8)
+        traffic = (None if args.separate_write or decode_only
+                   else profile_traffic(args.workload, fp8))
         probe = read_probe_gbs(torch, device) if args.read_probe else None
         swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe and not fp8 else None
         result = {
@@ -912,11 +949,12 @@ def run_pkv(args):
             "config": step_config(args, wl, npairs, pt_run, nbytes, scrub is not None, fp8),
             "roofline": {
                 "bound": "hbm",
-                "kernel": "%s (%sdecode + lse_reduce)" % (
-                    {(True, True): "kv_write_fp8_and_decode", (True, False):
-                     "paged_attn_decode_fp8", (False, True): "kv_write_and_decode",
-                     (False, False): "paged_attn_decode"}[(fp8, fused)],
-                    "newest-token write + " if fused else ""),
+                "kernel": ("attn_decode_contiguous (contiguous decode + lse_reduce)" if contig
+                           else "%s (%sdecode + lse_reduce)" % (
+                               {(True, True): "kv_write_fp8_and_decode", (True, False):
+                                "paged_attn_decode_fp8", (False, True): "kv_write_and_decode",
+                                (False, False): "paged_attn_decode"}[(fp8, fused)],
+                               "newest-token write + " if fused else "")),
                 "achieved": round(achieved, 1),
                 "peak": peak,
                 "peak_kind": peak_kind,
@@ -960,6 +998,9 @@ def run_pkv(args):
             result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
         if "sharing" in wl.extra:
             result["sharing"] = wl.extra["sharing"]
+        result["cache_bytes"] = {"paged_pools": 2 * kp.numel() * kp.element_size(),
+                                 "contiguous_reservation": (2 * kc.numel() * kc.element_size()
+                                                            if contig else None)}
         if defines:
             result["library"] = {"variant_defines": defines,
                                  "path": os.path.basename(os.environ["PKV_LIB"])}

@@ -161,6 +161,25 @@ pkv_status kv_write_and_decode(const pkv_attn_desc *desc, const void *q, const v
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Decode attention over a CONTIGUOUS cache, with no block table: the layout the paged cache
+ * replaces, kept as the baseline for the cost of the table ("vLLM and PagedAttention: How
+ * Ideas from Operating Systems Accelerated LLM Inference": the paged kernel ran 20-26 %
+ * slower than a contiguous one because of the block-table indirection).  Computes exactly
+ * what paged_attn_decode computes (same kernel body, same partitions and rounding), with
+ * token t of sequence s and kv head h at row t of a reservation of Lmax token rows:
+ *   k_cache/v_cache [S, H_kv, Lmax, D] dtype (f16 or bf16), 16-byte aligned, where
+ *                   Lmax = desc->max_blocks_per_seq * 16 (rows past context_lens[s] are
+ *                   never used)
+ *   context_lens    [S] int32, each in [1, Lmax] (checked on the device)
+ * q, out, scale, the workspace (pkv_attn_workspace_bytes(desc)) and the errors are as
+ * paged_attn_decode's; desc->num_blocks is not used.  S * H_kv * Lmax must stay below 2^31.
+ */
+pkv_status attn_decode_contiguous(const pkv_attn_desc *desc, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *context_lens, float scale,
+                                  void *out, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
  * Copy-on-write block copy ("Memory Optimization in LLM Serving with PagedAttention",
  * section "Advanced Capabilities: Memory Sharing with Copy-on-Write": before a sequence
  * writes into a block it shares, the block's content is copied to a fresh block).  For each

@@ -36,6 +36,7 @@ EXPORTS = [
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
     "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
     "kv_write_and_decode", "kv_write_fp8_and_decode", "pkv_fp8_partition_tokens",
+    "attn_decode_contiguous",
 ]
 
 
@@ -82,6 +83,7 @@ def lib():
         "kv_write_and_decode": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp,
                                  sz, vp], i32),
         "kv_copy_blocks": ([dp, vp, i32, vp, vp, vp], i32),
+        "attn_decode_contiguous": ([dp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz, vp], i32),
         "pkv_device_faults": ([P(ctypes.c_uint32), ctypes.c_int, vp], i32),
         "pkv_bm_create": ([i32, i32, vp, P(vp)], i32),
         "pkv_bm_destroy": ([vp], None),
@@ -224,6 +226,38 @@ def paged_attn_decode(q, k_pool, v_pool, block_tables, context_lens, scale, out=
                                    _ptr(block_tables), _ptr(context_lens), float(scale),
                                    _ptr(out), _ptr(workspace), nbytes,
                                    _stream(stream, q.device)))
+    return out
+
+
+def attn_decode_contiguous(q, k_cache, v_cache, context_lens, scale, out=None, workspace=None,
+                           partition_tokens=0, stream=None):
+    """The same decode over a contiguous cache with no block table: k_cache / v_cache
+    [S, H_kv, Lmax, D] (Lmax a multiple of 16), token t of sequence s at row t."""
+    _dev(q, "q")
+    _dev(k_cache, "k_cache", q.dtype)
+    _dev(v_cache, "v_cache", q.dtype)
+    _dev(context_lens, "context_lens", torch.int32)
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape or \
+            k_cache.shape[0] != q.shape[0] or k_cache.shape[3] != q.shape[2] or \
+            context_lens.shape != (q.shape[0],):
+        raise ValueError("q [S,Hq,D], caches [S,H_kv,Lmax,D], context_lens [S] expected")
+    S, Hq, D = q.shape
+    Hkv, lmax = k_cache.shape[1], k_cache.shape[2]
+    if lmax % BLOCK_SIZE:
+        raise ValueError("Lmax must be a multiple of %d" % BLOCK_SIZE)
+    desc = make_desc(S, Hq, Hkv, D, 1, lmax // BLOCK_SIZE, q.dtype, partition_tokens)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _dev(out, "out", q.dtype)
+    need = attn_workspace_bytes(desc)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().attn_decode_contiguous(ctypes.byref(desc), _ptr(q), _ptr(k_cache),
+                                        _ptr(v_cache), _ptr(context_lens), float(scale),
+                                        _ptr(out), _ptr(workspace), nbytes,
+                                        _stream(stream, q.device)))
     return out
 
 

@@ -87,6 +87,9 @@ struct DecodeParams {
     const void *k_new = nullptr;
     const void *v_new = nullptr;
     const int64_t *slot_mapping = nullptr;
+    // contiguous cache (attn_decode_contiguous): token rows per (sequence, kv head); 0 for
+    // the paged pools
+    int32_t Lmax = 0;
 };
 
 // Fused kv_write, called by the one warp per (sequence, kv head) that will copy the block

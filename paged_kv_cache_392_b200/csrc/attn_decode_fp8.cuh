@@ -32,14 +32,18 @@ __host__ __device__ __forceinline__ int v_slot_of_token(int t) {
     return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
 }
 
-// Two E4M3 codes (bytes 0 and 1 of w) to an f16x2 register holding each value times 2^-8,
-// with integer operations only: an E4M3 code s.eeee.mmm placed as the f16 s.0eeee.mmm0000000
-// is the same number scaled by 2^(7-15) = 2^-8, subnormals included (f16 keeps E4M3's
-// subnormal grid scaled by the same power of two).  byte << 8 puts s.eeee.mmm at bits
-// 15..8; subtracting ((x >> 1) & 0x3F80) moves eeee.mmm down one bit and keeps s.
+// Two E4M3 codes of w to an f16x2 register holding each value times 2^-8, with integer
+// operations only: an E4M3 code s.eeee.mmm placed as the f16 s.0eeee.mmm0000000 is the same
+// number scaled by 2^(7-15) = 2^-8, subnormals included (f16 keeps E4M3's subnormal grid
+// scaled by the same power of two).  A byte permute in sign-replicating mode builds
+// [sign(b_hi) x8 : b_hi : sign(b_lo) x8 : b_lo] (prmt selector nibbles with bit 3 set copy the
+// selected byte's sign bit into all 8 bits); shifted left by 7, each half holds eeee.mmm at
+// bits 13..7 and the sign at bit 15, and the mask keeps exactly those bits.  sel picks the
+// pair: 0x9180 for bytes 0 and 1, 0xB3A2 for bytes 2 and 3.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
-    const uint32_t t = __byte_perm(w, 0u, sel);  // [b_hi : 0 : b_lo : 0]
-    return t - ((t >> 1) & 0x3F803F80u);
+    uint32_t t;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
+    return (t << 7) & 0xBF80BF80u;
 }
 
 // How many of the 8 P.V m-tiles (16 head dims each) widen V on the conversion unit (XU
@@ -444,10 +448,10 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                     a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] & 0xffffu));
                     a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] >> 16));
                 } else {
-                    a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x1404u);
-                    a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x3424u);
-                    a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x1404u);
-                    a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x3424u);
+                    a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x9180u);
+                    a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0xB3A2u);
+                    a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x9180u);
+                    a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0xB3A2u);
                 }
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }

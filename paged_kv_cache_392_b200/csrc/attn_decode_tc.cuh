@@ -51,10 +51,13 @@ struct DecodeTcCfg {
     static_assert(G <= 8, "at most 8 query heads per kv head (one n=8 tile)");
 };
 
-template <typename T, int D, int G, int W, int NSW>
-__global__ void __launch_bounds__(W * 32)
-paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
-                            const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
+// The work of one CTA.  kContig false: the paged pools, block j of sequence s at physical
+// block block_tables[s][j], TMA row (phys * H_kv + hk) * 16.  kContig true: a contiguous cache
+// [S][H_kv][Lmax][D] with no block table, block j of sequence s at TMA row
+// (s * H_kv + hk) * Lmax + 16 j; everything else is the same code.
+template <typename T, int D, int G, int W, int NSW, bool kContig>
+__device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUtensorMap &tmv,
+                                               const DecodeParams &p) {
     using C = DecodeTcCfg<T, D, G, W, NSW>;
     constexpr bool BF = std::is_same<T, __nv_bfloat16>::value;
     constexpr int CHUNK = C::CHUNK, KSTEPS = C::KSTEPS, HALVES = C::HALVES, BOX = C::BOX;
@@ -104,27 +107,33 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
         }
     }
     __syncwarp();
-    if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
+    if (!kContig && p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
         write_newest_token<T, D>(p, s, hk, L, lane);
 
-    const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const int32_t *btrow = kContig ? nullptr : p.block_tables + (size_t)s * p.maxB + j0 + warp;
     const uint64_t policy = l2_evict_first_policy();
     int tab_chunk = 0;
-    int32_t tab = lane < nbw ? btrow[(size_t)W * lane] : 0;
+    int32_t tab = !kContig && lane < nbw ? btrow[(size_t)W * lane] : 0;
+    // contiguous cache: TMA row of this warp's first block
+    const int32_t crow0 = kContig ? (s * p.Hkv + hk) * p.Lmax + (j0 + warp) * kBlock : 0;
 
     // Issue block i of this warp into stage i % NSW: HALVES boxes of K, then of V.
     auto issue = [&](int i) {
-        if ((i >> 5) != tab_chunk) {
-            tab_chunk = i >> 5;
-            const int li = (tab_chunk << 5) + lane;
-            tab = li < nbw ? btrow[(size_t)W * li] : 0;
+        int32_t phys = 0;
+        if constexpr (!kContig) {
+            if ((i >> 5) != tab_chunk) {
+                tab_chunk = i >> 5;
+                const int li = (tab_chunk << 5) + lane;
+                tab = li < nbw ? btrow[(size_t)W * li] : 0;
+            }
+            phys = __shfl_sync(FULL, tab, i & 31);
         }
-        const int32_t phys = __shfl_sync(FULL, tab, i & 31);
         if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
-            if ((unsigned)phys < (unsigned)p.NB) {
-                const int32_t row = (phys * p.Hkv + hk) * kBlock;
+            if (kContig || (unsigned)phys < (unsigned)p.NB) {
+                const int32_t row = kContig ? crow0 + i * (W * kBlock)
+                                            : (phys * p.Hkv + hk) * kBlock;
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, 2 * CHUNK);
 #pragma unroll
@@ -321,6 +330,22 @@ paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
     }
     __syncthreads();
     merge_and_store<T, D, G, W>(p, mo, mml, s, hk, part, nparts);
+}
+
+template <typename T, int D, int G, int W, int NSW>
+__global__ void __launch_bounds__(W * 32)
+paged_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
+    decode_tc_body<T, D, G, W, NSW, false>(tmk, tmv, p);
+}
+
+// The same decode over a contiguous cache (no block table): the comparison kernel for the
+// cost of the table's indirection.
+template <typename T, int D, int G, int W, int NSW>
+__global__ void __launch_bounds__(W * 32)
+contiguous_attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmk,
+                                 const __grid_constant__ CUtensorMap tmv, const DecodeParams p) {
+    decode_tc_body<T, D, G, W, NSW, true>(tmk, tmv, p);
 }
 
 }  // namespace pkv

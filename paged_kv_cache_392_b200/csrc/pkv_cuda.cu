@@ -165,15 +165,17 @@ pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t str
 constexpr int kTcWarps = PKV_DECODE_TC_WARPS;
 constexpr int kTcStages = PKV_DECODE_TC_STAGES;
 
-// Tensor-core decode for 16-bit K/V.
-template <typename T, int D, int G>
+// Tensor-core decode for 16-bit K/V: the paged pools, or (kContig) a contiguous cache.
+template <typename T, int D, int G, bool kContig = false>
 pkv_status launch_decode_tc(const pkv::DecodeParams &prm, int32_t dtype, cudaStream_t stream) {
     using Cfg = pkv::DecodeTcCfg<T, D, G, kTcWarps, kTcStages>;
-    auto kern = pkv::paged_attn_decode_tc_kernel<T, D, G, kTcWarps, kTcStages>;
+    auto kern = kContig ? pkv::contiguous_attn_decode_tc_kernel<T, D, G, kTcWarps, kTcStages>
+                        : pkv::paged_attn_decode_tc_kernel<T, D, G, kTcWarps, kTcStages>;
     static std::atomic<bool> done[kMaxDevices];
     pkv_status st = ensure_smem(kern, Cfg::SMEM, done, "paged_attn_decode");
     if (st) return st;
-    const int64_t rows = (int64_t)prm.NB * prm.Hkv * pkv::kBlock;
+    const int64_t rows = kContig ? (int64_t)prm.S * prm.Hkv * prm.Lmax
+                                 : (int64_t)prm.NB * prm.Hkv * pkv::kBlock;
     CUtensorMap tmk, tmv;
     st = kv_tensor_map(&tmk, prm.k_pool, dtype, D, rows, "paged_attn_decode");
     if (st) return st;
@@ -212,14 +214,14 @@ bool use_tc(const pkv_attn_desc *d) {
 #endif
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kContig = false>
 pkv_status dispatch_group_tc(int g, const pkv::DecodeParams &prm, int32_t dtype,
                              cudaStream_t stream) {
     switch (g) {
-    case 1: return launch_decode_tc<T, D, 1>(prm, dtype, stream);
-    case 2: return launch_decode_tc<T, D, 2>(prm, dtype, stream);
-    case 4: return launch_decode_tc<T, D, 4>(prm, dtype, stream);
-    case 8: return launch_decode_tc<T, D, 8>(prm, dtype, stream);
+    case 1: return launch_decode_tc<T, D, 1, kContig>(prm, dtype, stream);
+    case 2: return launch_decode_tc<T, D, 2, kContig>(prm, dtype, stream);
+    case 4: return launch_decode_tc<T, D, 4, kContig>(prm, dtype, stream);
+    case 8: return launch_decode_tc<T, D, 8, kContig>(prm, dtype, stream);
     default: return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode: group %d", g);
     }
 }
@@ -426,6 +428,64 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
     dim3 grid((unsigned)(2 * num_pairs), (unsigned)slices);
     pkv::kv_copy_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
     return cuda_check(cudaGetLastError(), fn, "launch");
+}
+
+pkv_status attn_decode_contiguous(const pkv_attn_desc *desc, const void *q, const void *k_cache,
+                                  const void *v_cache, const int32_t *context_lens, float scale,
+                                  void *out, void *workspace, size_t workspace_bytes_given,
+                                  void *stream) {
+    const char *fn = "attn_decode_contiguous";
+    Split sp;
+    pkv_status st = check_attn_desc(desc, fn, &sp);
+    if (st) return st;
+    if (desc->dtype != PKV_F16 && desc->dtype != PKV_BF16)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: 16-bit caches only (f16, bf16)", fn);
+    const int64_t lmax = (int64_t)desc->max_blocks_per_seq * pkv::kBlock;
+    if ((int64_t)desc->num_seqs * desc->num_kv_heads * lmax >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_UNSUPPORTED, "%s: cache too large for 32-bit TMA rows", fn);
+    if (desc->num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !context_lens || !out)
+        return fail(PKV_ERR_INVALID, "%s: NULL tensor pointer", fn);
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(context_lens, 4))
+        return fail(PKV_ERR_INVALID, "%s: misaligned pointer", fn);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID, "%s: scale is not finite", fn);
+    const size_t need = workspace_bytes(desc, sp);
+    if (need) {
+        if (!workspace || workspace_bytes_given < need)
+            return fail(PKV_ERR_INVALID, "%s: workspace needs %zu bytes", fn, need);
+        if (!aligned(workspace, 256))
+            return fail(PKV_ERR_INVALID, "%s: workspace must be 256-byte aligned", fn);
+    }
+    pkv::DecodeParams prm;
+    prm.q = q;
+    prm.k_pool = k_cache;
+    prm.v_pool = v_cache;
+    prm.block_tables = nullptr;
+    prm.context_lens = context_lens;
+    prm.out = out;
+    const size_t rows = (size_t)desc->num_seqs * desc->num_q_heads * sp.pmax;
+    prm.ws_o = need ? static_cast<float *>(workspace) : nullptr;
+    prm.ws_ml = need ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 round_up(rows * desc->head_dim * 4, 256))
+                     : nullptr;
+    prm.S = desc->num_seqs;
+    prm.Hq = desc->num_q_heads;
+    prm.Hkv = desc->num_kv_heads;
+    prm.NB = desc->num_blocks;
+    prm.maxB = desc->max_blocks_per_seq;
+    prm.part_blocks = sp.part_blocks;
+    prm.pmax = sp.pmax;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.Lmax = (int32_t)lmax;
+    const int g = desc->num_q_heads / desc->num_kv_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (desc->dtype == PKV_F16)
+        return desc->head_dim == 64 ? dispatch_group_tc<__half, 64, true>(g, prm, PKV_F16, s)
+                                    : dispatch_group_tc<__half, 128, true>(g, prm, PKV_F16, s);
+    return desc->head_dim == 64
+               ? dispatch_group_tc<__nv_bfloat16, 64, true>(g, prm, PKV_BF16, s)
+               : dispatch_group_tc<__nv_bfloat16, 128, true>(g, prm, PKV_BF16, s);
 }
 
 }  // extern "C"

@@ -18,7 +18,8 @@ def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
-    return sorted({n for n in names if n.startswith(("pkv_", "paged_attn_decode", "kv_"))})
+    return sorted({n for n in names
+                   if n.startswith(("pkv_", "paged_attn_decode", "attn_decode", "kv_"))})
 
 
 @pytest.fixture(scope="module")
@@ -154,3 +155,20 @@ def test_fault_bits_agree_across_header_binding_and_kernels():
                                                 cuh)}
     assert header == kernels == set(B.FAULT_BITS)
     assert len(header) == 7
+
+
+def test_contiguous_decode_rejects_bad_arguments_before_launch(lib):
+    a = ctypes.c_void_p(1 << 20)
+    f = lib.attn_decode_contiguous
+    assert f(ctypes.byref(_desc(dtype=0, num_q_heads=2)), a, a, a, a, 0.1, a, None, 0,
+             None) == 3                                    # fp32: not built
+    assert f(ctypes.byref(_desc(num_seqs=0)), None, None, None, None, 0.1, None, None, 0,
+             None) == 0                                    # empty batch: nothing to do
+    assert f(ctypes.byref(_desc()), a, None, a, a, 0.1, a, None, 0, None) == 1
+    assert "NULL" in B.last_error()
+    big = _desc(num_seqs=4096, num_kv_heads=8, num_q_heads=8, max_blocks_per_seq=4096)
+    assert f(ctypes.byref(big), a, a, a, a, 0.1, a, None, 0, None) == 3
+    assert "32-bit" in B.last_error()
+    d2 = _desc(max_blocks_per_seq=100, partition_tokens=512)
+    assert f(ctypes.byref(d2), a, a, a, a, 0.1, a, None, 0, None) == 1
+    assert "workspace" in B.last_error()
