@@ -337,9 +337,18 @@ def kv_write(k_new, v_new, slot_mapping, k_pool, v_pool, stream=None):
                           _ptr(k_pool), _ptr(v_pool), _stream(stream, k_pool.device)))
 
 
+def _block_pools_desc(k_pool, v_pool):
+    """Descriptor for whole-block moves: 16-bit / fp32 pools, or FP8 pools (uint8, V stored
+    [NB, H_kv, D, 16]; a block's bytes are moved the same way)."""
+    if k_pool.dtype == torch.uint8:
+        NB, Hkv, Bs, D = _fp8_pools(k_pool, v_pool)
+        return make_desc(0, Hkv, Hkv, D, NB, 1, PKV_FP8_E4M3)
+    return _pool_desc(k_pool, v_pool)
+
+
 def kv_copy_blocks(src_dst_pairs, k_pool, v_pool, stream=None):
     """Block dst of both pools becomes a copy of block src, for each (src, dst) row."""
-    desc = _pool_desc(k_pool, v_pool)
+    desc = _block_pools_desc(k_pool, v_pool)
     _dev(src_dst_pairs, "src_dst_pairs", torch.int32)
     if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
         raise ValueError("src_dst_pairs must be [P, 2]")

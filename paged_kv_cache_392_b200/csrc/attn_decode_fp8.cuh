@@ -53,6 +53,12 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t 
 #endif
 constexpr int kCvtTiles = PKV_FP8_CVT_TILES;
 
+// 1: a warp returns a stage to the copy engine as soon as the block is in its registers,
+// before the math (two blocks in flight during the math); 0: after the math.
+#ifndef PKV_FP8_EARLY_RELEASE
+#define PKV_FP8_EARLY_RELEASE 1
+#endif
+
 // Two E4M3 codes (low byte first) to an f16x2 register, exactly, on the conversion unit.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
     __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
@@ -368,18 +374,39 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             __syncwarp();
         }
 
-        // ---- S^T = K Q^T on E4M3 tiles: K codes go from ldmatrix straight into the A
-        // fragments (row g / g+8, k 4tq..4tq+3 and 16+4tq..16+4tq+3 of each 32-dim step)
-        // the high and residual q terms accumulate separately: two MMA chains of K32
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sres[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- the whole stage into registers: the K codes as the A fragments of S^T (row
+        // g / g+8, k 4tq..4tq+3 and 16+4tq..16+4tq+3 of each 32-dim step) and the V^T rows
+        // (r[0]: dims 32t2+0..7, r[1]: +8..15 of m-tile 2t2; r[2], r[3]: m-tile 2t2+1)
+        uint32_t ka[K32][4], vr[KSTEPS / 2][4];
         const uint32_t kb = smem_u32(Ks);
 #pragma unroll
         for (int j = 0; j < K32; ++j) {
             const int c = 2 * j + k_c;  // 16-byte chunk of the 128-byte row
-            uint32_t a[4];
-            ldmatrix_x4(a, kb + k_tok * 128 + ((c ^ (k_tok & 7)) << 4));
-            mma_16832_e4m3(sacc, a, qhi[j][0], qhi[j][1]);
-            mma_16832_e4m3(sres, a, qlo[j][0], qlo[j][1]);
+            ldmatrix_x4(ka[j], kb + k_tok * 128 + ((c ^ (k_tok & 7)) << 4));
+        }
+        const uint32_t vb = smem_u32(Vs);
+#pragma unroll
+        for (int t2 = 0; t2 < KSTEPS / 2; ++t2) ldmatrix_x4(vr[t2], vb + (32 * t2 + v_row) * 16);
+#if PKV_FP8_EARLY_RELEASE
+        // The stage now lives in registers: hand it back to the copy engine before the math,
+        // so that two blocks stay in flight while this one is computed (a stage refilled only
+        // after its math leaves one, and the warp waits on memory).  Every lane orders its
+        // shared-memory reads before the copy that overwrites them.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (issued < nbw) {
+            issue(issued);
+            ++issued;
+        }
+#endif
+
+        // ---- S^T = K Q^T on E4M3 tiles; the high and residual q terms accumulate separately:
+        // two MMA chains of K32
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sres[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < K32; ++j) {
+            mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
+            mma_16832_e4m3(sres, ka[j], qlo[j][0], qlo[j][1]);
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
@@ -433,12 +460,9 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         const uint32_t b1 = movmatrix_trans(f32x2_to_f16x2(p2, p3));
 
         // ---- O^T += V^T P^T -----------------------------------------------------------------
-        const uint32_t vb = smem_u32(Vs);
 #pragma unroll
         for (int t2 = 0; t2 < KSTEPS / 2; ++t2) {
-            uint32_t r[4];
-            ldmatrix_x4(r, vb + (32 * t2 + v_row) * 16);
-            // r[0]: dims 32t2+0..7, r[1]: +8..15 (m-tile 2t2); r[2], r[3]: m-tile 2t2+1
+            const uint32_t(&r)[4] = vr[t2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t a[4];
@@ -456,12 +480,13 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }
         }
+#if !PKV_FP8_EARLY_RELEASE
         __syncwarp();
-
         if (issued < nbw) {
             issue(issued);
             ++issued;
         }
+#endif
     }
     if (dead) {
         for (int b = i; b < issued; ++b)
