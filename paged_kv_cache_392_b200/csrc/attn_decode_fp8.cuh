@@ -48,16 +48,11 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t 
 
 // How many of the 8 P.V m-tiles (16 head dims each) widen V on the conversion unit (XU
 // pipe, exact values); the others use the integer trick above (ALU pipe, values x 2^-8).
+// With the three-operation integer form, none on the conversion unit measured fastest.
 #ifndef PKV_FP8_CVT_TILES
-#define PKV_FP8_CVT_TILES 4
+#define PKV_FP8_CVT_TILES 0
 #endif
 constexpr int kCvtTiles = PKV_FP8_CVT_TILES;
-
-// 1: a warp returns a stage to the copy engine as soon as the block is in its registers,
-// before the math (two blocks in flight during the math); 0: after the math.
-#ifndef PKV_FP8_EARLY_RELEASE
-#define PKV_FP8_EARLY_RELEASE 1
-#endif
 
 // Two E4M3 codes (low byte first) to an f16x2 register, exactly, on the conversion unit.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
@@ -263,13 +258,20 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     // terms, hi = e4m3(q*qf) and lo = e4m3(q*qf - hi), which carry about 8 significant bits
     // (a bfloat16 q exactly, up to subnormal tails).  Lane (g, tq) holds head g, dims
     // 32j+4tq..+3 (b0) and 32j+16+4tq..+3 (b1) of k-step j.
+    // With at most four query heads per kv head the two terms share one MMA chain: column n
+    // of the B operand holds the high term of head n (n < G) or the residual of head n - G
+    // (G <= n < 2G), and the two columns of a head are added after the chain.  Each column's
+    // sum is the one the separate chains computed, so the scores are the same bits; the
+    // E4M3 tiles cost about a dozen instructions each on this path, and this halves them.
     constexpr int K32 = D / 32;
+    constexpr bool kPack = G <= 4;
     uint32_t qhi[K32][2], qlo[K32][2];
     float qf_mine = 1.f;
     {
-        const bool hv = g < G;
+        const bool hv = kPack ? g < 2 * G : g < G;
+        const int qh = kPack && g >= G ? g - G : g;  // head of this lane's B column
         const T *qrow =
-            static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
+            static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? qh : 0)) * D;
         float qv[K32][2][4];
         float amax = 0.f;
 #pragma unroll
@@ -314,7 +316,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                     hi |= static_cast<uint32_t>(h2) << (8 * e);
                     lo |= static_cast<uint32_t>(l2) << (8 * e);
                 }
-                qhi[j][b] = hi;
+                qhi[j][b] = kPack && g >= G ? lo : hi;
                 qlo[j][b] = lo;
             }
     }
@@ -387,29 +389,30 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         const uint32_t vb = smem_u32(Vs);
 #pragma unroll
         for (int t2 = 0; t2 < KSTEPS / 2; ++t2) ldmatrix_x4(vr[t2], vb + (32 * t2 + v_row) * 16);
-#if PKV_FP8_EARLY_RELEASE
-        // The stage now lives in registers: hand it back to the copy engine before the math,
-        // so that two blocks stay in flight while this one is computed (a stage refilled only
-        // after its math leaves one, and the warp waits on memory).  Every lane orders its
-        // shared-memory reads before the copy that overwrites them.
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (issued < nbw) {
-            issue(issued);
-            ++issued;
-        }
-#endif
 
-        // ---- S^T = K Q^T on E4M3 tiles; the high and residual q terms accumulate separately:
-        // two MMA chains of K32
-        float sacc[4] = {0.f, 0.f, 0.f, 0.f}, sres[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- S^T = K Q^T on E4M3 tiles: the high and residual q terms in one chain of K32
+        // (packed columns, G <= 4), or in two
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (kPack) {
 #pragma unroll
-        for (int j = 0; j < K32; ++j) {
-            mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
-            mma_16832_e4m3(sres, ka[j], qlo[j][0], qlo[j][1]);
+            for (int j = 0; j < K32; ++j) mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
+            if constexpr (G == 1) {  // columns 0 (high) and 1 (residual) sit in one lane
+                sacc[0] += sacc[1];
+                sacc[2] += sacc[3];
+            } else {                 // the residual columns sit G/2 lanes (G columns) away
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[e] += __shfl_xor_sync(FULL, sacc[e], G / 2);
+            }
+        } else {
+            float sres[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < K32; ++j) {
+                mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
+                mma_16832_e4m3(sres, ka[j], qlo[j][0], qlo[j][1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
 
         // ---- online softmax (lane: tokens g, g+8 of heads 2tq, 2tq+1) --------------------
         float x0 = sacc[0] * sl0, x1 = sacc[1] * sl1, x2 = sacc[2] * sl0, x3 = sacc[3] * sl1;
@@ -480,13 +483,11 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }
         }
-#if !PKV_FP8_EARLY_RELEASE
         __syncwarp();
         if (issued < nbw) {
             issue(issued);
             ++issued;
         }
-#endif
     }
     if (dead) {
         for (int b = i; b < issued; ++b)
