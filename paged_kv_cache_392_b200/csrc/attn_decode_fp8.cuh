@@ -43,8 +43,25 @@ __host__ __device__ __forceinline__ int v_slot_of_token(int t) {
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
     uint32_t t;
     asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
+#if PKV_FP8_WIDEN_MUL
+    // the shift as a multiply, which the FMA pipe can take
+    uint32_t u;
+    asm("mul.lo.u32 %0, %1, 128;" : "=r"(u) : "r"(t));
+    return u & 0xBF80BF80u;
+#else
     return (t << 7) & 0xBF80BF80u;
+#endif
 }
+
+// Tuning switches of the FP8 decode (results are the same bits either way):
+//   PKV_FP8_SPEC_EXP 1: the softmax weights are computed before the rescale vote resolves
+//   PKV_FP8_WIDEN_MUL 1: the widening's shift is written as a multiply (FMA pipe)
+#ifndef PKV_FP8_SPEC_EXP
+#define PKV_FP8_SPEC_EXP 1
+#endif
+#ifndef PKV_FP8_WIDEN_MUL
+#define PKV_FP8_WIDEN_MUL 0
+#endif
 
 // How many of the 8 P.V m-tiles (16 head dims each) widen V on the conversion unit (XU
 // pipe, exact values); the others use the integer trick above (ALU pipe, values x 2^-8).
@@ -427,6 +444,12 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         // does not depend on the reference.  One vote tells whether any score passes its
         // reference by that much; only then (a warp's first block, and rarely after) does
         // the warp reduce the block's max and rescale O and its partial sums.
+#if PKV_FP8_SPEC_EXP
+        // The weights against the current references start before the vote resolves; the
+        // rare block that moves a reference computes them again.
+        float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
+        float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         if (__any_sync(FULL, fmaxf(x0, x2) > m_run[0] + kLazyRescale ||
                                  fmaxf(x1, x3) > m_run[1] + kLazyRescale)) {
             float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
@@ -450,9 +473,17 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             }
             m_run[0] = mn0;
             m_run[1] = mn1;
+#if PKV_FP8_SPEC_EXP
+            p0 = ex2_ftz(x0 - m_run[0]);
+            p1 = ex2_ftz(x1 - m_run[1]);
+            p2 = ex2_ftz(x2 - m_run[0]);
+            p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         }
+#if !PKV_FP8_SPEC_EXP
         const float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
         const float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         // per-lane partial sums; the 8 token-row lanes of a head add theirs after the loop
         l_run[0] += p0 + p2;
         l_run[1] += p1 + p3;
