@@ -33,6 +33,12 @@
 #ifndef PKV_DECODE_TC_STAGES
 #define PKV_DECODE_TC_STAGES 2
 #endif
+// 1: the softmax weights are computed before the rescale vote resolves, as in the FP8
+// decode (the same bits either way; measured +1.4 / +1.7 % on the fork / beam steps, within
+// noise elsewhere).
+#ifndef PKV_TC_SPEC_EXP
+#define PKV_TC_SPEC_EXP 1
+#endif
 
 namespace pkv {
 
@@ -233,6 +239,12 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
         // depend on the reference.  One vote tells whether any score passes its reference
         // by that much; only then (a warp's first block, and rarely after) does the warp
         // reduce the block's max and rescale O and its partial sums.
+#if PKV_TC_SPEC_EXP
+        // The weights against the current references start before the vote resolves; the
+        // rare block that moves a reference computes them again.
+        float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
+        float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         if (__any_sync(FULL, fmaxf(x0, x2) > m_run[0] + kLazyRescale ||
                                  fmaxf(x1, x3) > m_run[1] + kLazyRescale)) {
             float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
@@ -256,9 +268,17 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
             }
             m_run[0] = mn0;
             m_run[1] = mn1;
+#if PKV_TC_SPEC_EXP
+            p0 = ex2_ftz(x0 - m_run[0]);
+            p1 = ex2_ftz(x1 - m_run[1]);
+            p2 = ex2_ftz(x2 - m_run[0]);
+            p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         }
+#if !PKV_TC_SPEC_EXP
         const float p0 = ex2_ftz(x0 - m_run[0]), p1 = ex2_ftz(x1 - m_run[1]);
         const float p2 = ex2_ftz(x2 - m_run[0]), p3 = ex2_ftz(x3 - m_run[1]);
+#endif
         // per-lane partial sums; the 8 token-row lanes of a head add theirs after the loop
         l_run[0] += p0 + p2;
         l_run[1] += p1 + p3;
