@@ -565,12 +565,15 @@ int device_sm_count() {
 // default 512.  Measured on the OPT-13B-shaped batch: +13 %.  Never more partitions than the
 // default, so the default's workspace always suffices.
 constexpr int32_t kFp8WidePartitionTokens = 2048;
+// Resident warps per SM the choice counts with (fixed, so that the partition, and with it the
+// rounding of the result, does not change when the kernel's occupancy is tuned).
+constexpr int kFp8PartitionWarpsPerSm = 16;
 
 Split fp8_split(const pkv_attn_desc *d, const Split &dflt) {
     if (d->partition_tokens != 0) return dflt;
     const int g = d->num_q_heads / d->num_kv_heads;
     const int warps = g == 1 ? fp8_warps<1>() : fp8_warps<2>();
-    const int64_t slots = (int64_t)device_sm_count() * (pkv::kFp8WarpsPerSm / warps);
+    const int64_t slots = (int64_t)device_sm_count() * (kFp8PartitionWarpsPerSm / warps);
     const int64_t pairs = (int64_t)d->num_seqs * d->num_kv_heads;
     if (slots <= 0 || pairs < 4 * slots) return dflt;
     Split sp;
