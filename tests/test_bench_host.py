@@ -7,6 +7,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
@@ -116,3 +117,41 @@ def test_split_rows_counts_only_sequences_that_span_partitions():
     rows, pmax = bench.split_rows(wl, 16)
     assert pmax == 3 and rows == (2 + 3 + 3) * wl.num_q_heads
     assert bench.split_rows(wl, 0) == (0, 1)
+
+
+def _fake_workload(lens, tables):
+    class _W:
+        pass
+    w = _W()
+    w.context_lens = np.asarray(lens, np.int32)
+    w.block_tables = np.asarray(tables, np.int32)
+    return w
+
+
+def test_kv_utilisation_follows_the_pages_waste_examples():
+    """The pages' worked examples (300 and 50 tokens in 16-token blocks): slots allocated and
+    filled as the fixture states; a block that two sequences map counts once."""
+    golden = json.load(open(os.path.join(ROOT, "tests", "golden", "waste_examples.json")))
+    for c in golden["cases"]:
+        nb = c["paged_blocks"]
+        u = bench.kv_utilisation(_fake_workload([c["tokens"]], [list(range(nb))]))
+        assert u["slots_allocated"] == c["paged_slots"]
+        assert u["slots_allocated"] - u["tokens_in_blocks"] == c["paged_wasted"]
+    # two sequences sharing a full first block: 16 + 5 + 9 tokens in 3 distinct blocks
+    u = bench.kv_utilisation(_fake_workload([21, 25], [[7, 3], [7, 4]]))
+    assert u["slots_allocated"] == 48 and u["tokens_in_blocks"] == 16 + 5 + 9
+
+
+def test_both_arms_describe_the_step_with_one_config():
+    args = bench.parse_args(["--workload", "fork"])
+    wl, pairs = bench.build_workload("fork")
+    wl2, pairs2 = bench.build_workload("fork", model_block_manager=True)
+    assert np.array_equal(wl.block_tables, wl2.block_tables)
+    assert np.array_equal(pairs, pairs2)
+    rows, _ = bench.split_rows(wl, 512)
+    nb = bench.algorithmic_bytes(wl, pairs, rows)
+    c1 = bench.step_config(args, wl, len(pairs), 512, nb, bench.uses_l2_flush(args, wl, nb, False),
+                           False)
+    c2 = bench.step_config(args, wl2, len(pairs2), 512, nb,
+                           bench.uses_l2_flush(args, wl2, nb, False), False)
+    assert c1 == c2 and c1["cow_pairs_per_step"] == 112
