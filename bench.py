@@ -383,14 +383,23 @@ DECODE_SOURCES = ("attn_decode.cuh", "attn_decode_tc.cuh", "ptx.cuh", "faults.cu
 DECODE_FP8_SOURCES = DECODE_SOURCES + ("attn_decode_fp8.cuh", "pkv_cuda.cu")
 
 
+def _code_only(text):
+    """Source text without comments, trailing spaces and blank lines: what the compiler sees
+    of it (the kernel sources hold no comment markers inside string literals)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def kernel_source_sha(fp8=False):
-    """Hash of the decode kernels' sources (kernels and their launch shape); the FP8 kernel's
-    launch constants live in the launcher, so its hash covers that file too."""
+    """Hash of the decode kernels' code (kernels and their launch shape; comments left out);
+    the FP8 kernel's launch constants live in the launcher, so its hash covers that file
+    too."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc")
     for name in (DECODE_FP8_SOURCES if fp8 else DECODE_SOURCES):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

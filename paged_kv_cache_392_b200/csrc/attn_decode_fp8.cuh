@@ -12,10 +12,11 @@
 //     the 4 bytes an ldmatrix lane reads from a row are the token pairs the P.V tile wants.
 // Decode: q.K^T runs on m16n8k32 E4M3 tensor-core tiles straight from the K codes, with each
 // query row prescaled by a power of two and split into two E4M3 terms (hi + residual, about
-// bfloat16 precision); P.V widens the V codes exactly to f16 (every E4M3 value is an f16
-// value; half of the tiles on the integer pipe, half on the conversion unit) for m16n8k16
-// f16 tiles.  Accumulation is fp32; the K scale (and the q prescale) is folded into the
-// softmax scale and the V scale into the output.  Only D = 128 is built.
+// bfloat16 precision; with at most four query heads per kv head both terms ride in one MMA
+// chain, side by side in the n columns); P.V widens the V codes exactly to f16 (every E4M3
+// value is an f16 value, scaled by 2^-8 on the integer path) for m16n8k16 f16 tiles.
+// Accumulation is fp32; the K scale (and the q prescale) is folded into the softmax scale
+// and the V scale into the output.  Only D = 128 is built.
 #pragma once
 #include <cuda.h>
 #include <cuda_fp8.h>
