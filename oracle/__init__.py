@@ -217,15 +217,23 @@ def f32_to_e4m3(x: float) -> int:
     return int(lib().orc_f32_to_e4m3(float(x)))
 
 
+def _fp8_v_shape_ok(v_pool, NB, Hkv, B, D):
+    """FP8 V pools: [NB, Hkv, B/16, D, 16] (each 16-token half of a block transposed), which
+    for B = 16 may also be given as [NB, Hkv, D, 16]."""
+    return v_pool.shape == (NB, Hkv, B // 16, D, 16) or (B == 16 and v_pool.shape ==
+                                                          (NB, Hkv, D, 16))
+
+
 def kv_write_fp8(k_new, v_new, slot_mapping, k_scale, v_scale, k_pool, v_pool, dtype):
     """Quantise new K/V rows [T, Hkv, D] of ``dtype`` into uint8 E4M3 pools, in place:
-    K pool [NB, Hkv, B, D], V pool [NB, Hkv, D, B] (transposed within the block; slot p of
-    a row holds token 2*(p//4) + p%2 + 8*((p//2)%2))."""
+    K pool [NB, Hkv, B, D]; V pool [NB, Hkv, B/16, D, 16]: each 16-token half of a block
+    transposed, slot p of a row holding token 2*(p//4) + p%2 + 8*((p//2)%2) of the half
+    ([NB, Hkv, D, 16] when B = 16)."""
     k_new = _as_bits(k_new, dtype)
     v_new = _as_bits(v_new, dtype)
     T, Hkv, D = k_new.shape
     NB, Hkv2, B, D2 = k_pool.shape
-    if (Hkv2, D2) != (Hkv, D) or v_pool.shape != (NB, Hkv, D, B):
+    if (Hkv2, D2) != (Hkv, D) or not _fp8_v_shape_ok(v_pool, NB, Hkv, B, D):
         raise ValueError("shape mismatch")
     for a in (k_pool, v_pool):
         if a.dtype != np.uint8 or not a.flags.c_contiguous:
@@ -244,7 +252,7 @@ def paged_attn_decode_fp8(q, k_pool, v_pool, k_scale, v_scale, block_tables, con
     q = _as_bits(q, q_dtype)
     S, Hq, D = q.shape
     NB, Hkv, B, D2 = k_pool.shape
-    if D2 != D or v_pool.shape != (NB, Hkv, D, B):
+    if D2 != D or not _fp8_v_shape_ok(v_pool, NB, Hkv, B, D):
         raise ValueError("shape mismatch")
     bt = np.ascontiguousarray(block_tables, dtype=np.int32)
     lens = np.ascontiguousarray(context_lens, dtype=np.int32)

@@ -400,15 +400,26 @@ static float orc_load_f32(const void *base, int dtype, size_t i) {
 }
 
 /*
- * kv_write into FP8 pools: for token t and head h with slot s (s = -1 skips),
+ * Byte offset of token `off` (of a B-token block), dim d, in the FP8 V pool
+ * [NB][Hkv][B/16][D][16]: every 16-token half of a block is stored transposed, its row of
+ * 16 slots in the slot order above.  With B = 16 this is [NB][Hkv][D][16].
+ */
+static size_t orc_v_fp8_index(int64_t blk, int h, int off, int d, int Hkv, int B, int D) {
+    return ((((size_t)blk * Hkv + h) * (size_t)(B / 16) + (size_t)(off / 16)) * D + d) * 16 +
+           (size_t)orc_v_slot(off % 16);
+}
+
+/*
+ * kv_write into FP8 pools (B a multiple of 16): for token t and head h with slot s
+ * (s = -1 skips),
  *   k_pool[s/B][h][s%B][d] = e4m3(k_new[t][h][d] / k_scale[h])
- *   v_pool[s/B][h][d][s%B] = e4m3(v_new[t][h][d] / v_scale[h])
+ *   v_pool at orc_v_fp8_index(s/B, h, s%B, d) = e4m3(v_new[t][h][d] / v_scale[h])
  */
 int orc_kv_write_fp8(int T, int Hkv, int D, int B, int NB, const void *k_new,
                      const void *v_new, int new_dtype, const int64_t *slot_mapping,
                      const float *k_scale, const float *v_scale, uint8_t *k_pool,
                      uint8_t *v_pool) {
-    if (T < 0 || Hkv < 1 || D < 1 || B != 16 || NB < 0 || !orc_elem_size(new_dtype))
+    if (T < 0 || Hkv < 1 || D < 1 || B < 16 || B % 16 || NB < 0 || !orc_elem_size(new_dtype))
         return ORC_BAD_ARG;
     int err = ORC_OK;
     for (int t = 0; t < T; ++t) {
@@ -423,8 +434,7 @@ int orc_kv_write_fp8(int T, int Hkv, int D, int B, int NB, const void *k_new,
                 float kq = orc_load_f32(k_new, new_dtype, src) / k_scale[h];
                 float vq = orc_load_f32(v_new, new_dtype, src) / v_scale[h];
                 k_pool[(((size_t)blk * Hkv + h) * B + off) * D + d] = orc_f32_to_e4m3(kq);
-                v_pool[(((size_t)blk * Hkv + h) * D + d) * B + orc_v_slot(off)] =
-                    orc_f32_to_e4m3(vq);
+                v_pool[orc_v_fp8_index(blk, h, off, d, Hkv, B, D)] = orc_f32_to_e4m3(vq);
             }
     }
     return err;
@@ -438,8 +448,8 @@ int orc_paged_attn_decode_fp8(int S, int Hq, int Hkv, int D, int B, int NB, int 
                               const float *v_scale, const int32_t *block_tables,
                               const int32_t *context_lens, double scale, const int32_t *rows,
                               int nrows, double *out, int nthreads) {
-    if (S < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || B != 16 || NB < 0 || maxB < 0 ||
-        !orc_elem_size(q_dtype))
+    if (S < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || B < 16 || B % 16 || NB < 0 ||
+        maxB < 0 || !orc_elem_size(q_dtype))
         return ORC_BAD_ARG;
     int n = rows ? nrows : S * Hq;
     int err = ORC_OK;
@@ -478,8 +488,7 @@ int orc_paged_attn_decode_fp8(int S, int Hq, int Hkv, int D, int B, int NB, int 
             den += w;
             for (int d = 0; d < D; ++d)
                 o[d] += w * (orc_e4m3_to_f64(
-                                 v_pool[(((size_t)p * Hkv + hk) * D + d) * B + orc_v_slot(t % B)]) *
-                             vs);
+                                 v_pool[orc_v_fp8_index(p, hk, t % B, d, Hkv, B, D)]) * vs);
         }
         for (int d = 0; d < D; ++d) o[d] /= den;
         free(x);

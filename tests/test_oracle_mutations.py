@@ -36,8 +36,13 @@ MUTATIONS = {
     "e4m3 encoder truncates": ("int n = (int)nearbyint(a / ldexp(1.0, e - 3));",
                                "int n = (int)floor(a / ldexp(1.0, e - 3));"),
     "fp8 V written untransposed": (
-        "v_pool[(((size_t)blk * Hkv + h) * D + d) * B + orc_v_slot(off)] =",
-        "v_pool[(((size_t)blk * Hkv + h) * B + orc_v_slot(off)) * D + d] ="),
+        "return ((((size_t)blk * Hkv + h) * (size_t)(B / 16) + (size_t)(off / 16)) * D + d) * 16 +\n"
+        "           (size_t)orc_v_slot(off % 16);",
+        "return ((((size_t)blk * Hkv + h) * (size_t)(B / 16) + (size_t)(off / 16)) * 16 +\n"
+        "           (size_t)orc_v_slot(off % 16)) * D + d;"),
+    "fp8 V halves of a 32-token block swapped": (
+        "(size_t)(B / 16) + (size_t)(off / 16)) * D + d) * 16 +",
+        "(size_t)(B / 16) + (size_t)((B / 16 - 1) - off / 16)) * D + d) * 16 +"),
     "fp8 V slot order ignored": ("if (2 * (p / 4) + p % 2 + 8 * ((p / 2) % 2) == t) return p;",
                                  "if (p == t) return p;"),
     "fp8 K scale dropped": ("(orc_e4m3_to_f64(k_pool[(((size_t)p * Hkv + hk) * B + t % B) * D + d]) * ks)",
@@ -49,7 +54,8 @@ MUTATIONS = {
 PINS = [
     pins.test_f16_decoder_matches_ieee_binary16_for_all_patterns,
     pins.test_bf16_decoder_matches_upper_half_of_binary32_for_all_patterns,
-    lambda: pins.test_oracle_matches_bruteforce_contiguous_attention(4, 2, 32),
+    lambda: pins.test_oracle_matches_bruteforce_contiguous_attention(4, 2, 32, 16),
+    lambda: pins.test_oracle_matches_bruteforce_contiguous_attention(4, 2, 32, 32),
     pins.test_oracle_matches_torch_sdpa_fp64_on_contiguous_layout,
     pins.test_oracle_16bit_inputs_match_bruteforce_on_upcast_values,
     pins.test_golden_closed_form_example,
@@ -62,8 +68,10 @@ PINS = [
     pins.test_kv_copy_blocks_copies_whole_blocks,
     pins8.test_e4m3_decoder_matches_torch_for_all_codes,
     pins8.test_e4m3_encoder_matches_torch_rounding_in_range,
-    pins8.test_kv_write_fp8_quantises_into_the_two_layouts,
-    pins8.test_fp8_decode_matches_bruteforce_on_dequantised_values,
+    lambda: pins8.test_kv_write_fp8_quantises_into_the_two_layouts(16),
+    lambda: pins8.test_kv_write_fp8_quantises_into_the_two_layouts(32),
+    lambda: pins8.test_fp8_decode_matches_bruteforce_on_dequantised_values(16),
+    lambda: pins8.test_fp8_decode_matches_bruteforce_on_dequantised_values(32),
 ]
 
 

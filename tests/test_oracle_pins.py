@@ -83,11 +83,12 @@ def _brute(q, kc, vc, scale, Hq, Hkv):
 
 
 # ---------------------------------------------------------------- brute force / library
-@pytest.mark.parametrize("Hq,Hkv,D", [(2, 2, 64), (4, 2, 32), (8, 1, 16)])
-def test_oracle_matches_bruteforce_contiguous_attention(Hq, Hkv, D):
+@pytest.mark.parametrize("Hq,Hkv,D,B", [(2, 2, 64, 16), (4, 2, 32, 16), (8, 1, 16, 16),
+                                        (4, 2, 32, 32)])
+def test_oracle_matches_bruteforce_contiguous_attention(Hq, Hkv, D, B):
     rng = np.random.default_rng(11)
-    lens = [1, 5, 15, 16, 17, 33, 48, 70]
-    q, kc, vc, kp, vp, bt = _rand_case(rng, lens, Hq, Hkv, D)
+    lens = [1, 5, 15, 16, 17, 31, 32, 33, 48, 70]
+    q, kc, vc, kp, vp, bt = _rand_case(rng, lens, Hq, Hkv, D, B=B)
     scale = 1.0 / math.sqrt(D)
     got = oracle.paged_attn_decode(q, kp, vp, bt, np.array(lens, np.int32), scale, "f32")
     ref = _brute(q, kc, vc, scale, Hq, Hkv)

@@ -43,15 +43,16 @@ def test_e4m3_encoder_saturates_and_keeps_nan():
     assert oracle.f32_to_e4m3(-0.0) == 0x80 and oracle.f32_to_e4m3(0.0) == 0x00
 
 
-def test_kv_write_fp8_quantises_into_the_two_layouts():
+@pytest.mark.parametrize("B", [16, 32])
+def test_kv_write_fp8_quantises_into_the_two_layouts(B):
     rng = np.random.default_rng(1)
-    NB, Hkv, B, D, T = 5, 2, 16, 8, 3
+    NB, Hkv, D, T = 5, 2, 8, 3
     kn = torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).half()
     vn = torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).half()
     ks = np.array([0.01, 0.02], np.float32)
     vs = np.array([0.03, 0.005], np.float32)
     kp = np.zeros((NB, Hkv, B, D), np.uint8)
-    vp = np.zeros((NB, Hkv, D, B), np.uint8)
+    vp = np.zeros((NB, Hkv, B // 16, D, 16), np.uint8)     # each 16-token half transposed
     slots = np.array([17, -1, 79], np.int64)
     bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
     oracle.kv_write_fp8(bits(kn), bits(vn), slots, ks, vs, kp, vp, "f16")
@@ -64,23 +65,24 @@ def test_kv_write_fp8_quantises_into_the_two_layouts():
         if sl < 0:
             continue
         blk, off = sl // B, sl % B
-        vslot = token_of_slot.index(off)
+        vslot = token_of_slot.index(off % 16)
         for h in range(Hkv):
             qk = torch.from_numpy(kn[t, h].float().numpy() / ks[h]).to(torch.float8_e4m3fn)
             qv = torch.from_numpy(vn[t, h].float().numpy() / vs[h]).to(torch.float8_e4m3fn)
             ek[blk, h, off, :] = qk.view(torch.uint8).numpy()
-            ev[blk, h, :, vslot] = qv.view(torch.uint8).numpy()
+            ev[blk, h, off // 16, :, vslot] = qv.view(torch.uint8).numpy()
     assert np.array_equal(kp, ek) and np.array_equal(vp, ev)
 
 
-def test_fp8_decode_matches_bruteforce_on_dequantised_values():
+@pytest.mark.parametrize("B", [16, 32])
+def test_fp8_decode_matches_bruteforce_on_dequantised_values(B):
     rng = np.random.default_rng(2)
-    Hq, Hkv, D, B = 8, 2, 32, 16
-    lens = [1, 15, 16, 17, 40, 70]
+    Hq, Hkv, D = 8, 2, 32
+    lens = [1, 15, 16, 17, 31, 32, 33, 40, 70]
     nblk = [-(-L // B) for L in lens]
     NB = sum(nblk) + 2
     kp = rng.integers(0, 256, (NB, Hkv, B, D), dtype=np.uint8)
-    vp = rng.integers(0, 256, (NB, Hkv, D, B), dtype=np.uint8)
+    vp = rng.integers(0, 256, (NB, Hkv, B // 16, D, 16), dtype=np.uint8)
     kp[(kp & 0x7F) == 0x7F] = 0x10              # no NaN codes
     vp[(vp & 0x7F) == 0x7F] = 0x10
     ks = rng.uniform(0.001, 0.01, Hkv).astype(np.float32)
@@ -101,7 +103,8 @@ def test_fp8_decode_matches_bruteforce_on_dequantised_values():
         for h in range(Hq):
             hk = h // g
             K = np.array([table[kp[bt[s, t // B], hk, t % B, :]] for t in range(L)]) * ks[hk]
-            V = np.array([table[vp[bt[s, t // B], hk, :, token_of_slot.index(t % B)]]
+            V = np.array([table[vp[bt[s, t // B], hk, (t % B) // 16, :,
+                                   token_of_slot.index(t % 16)]]
                           for t in range(L)]) * vs[hk]
             x = K @ q[s, h].astype(np.float64) * 0.2
             w = np.exp(x - x.max())
