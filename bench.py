@@ -85,6 +85,9 @@ def parse_args(argv=None):
                     help="contiguous: time attn_decode_contiguous over a [S][H_kv][Lmax][D] "
                          "cache with no block table (the same tokens, gathered from the "
                          "pools), decode only; compare with --decode-only on the paged pools")
+    ap.add_argument("--block-size", type=int, default=16, choices=[16, 32],
+                    help="tokens per physical KV block (opt13b, gqa, long); the configs "
+                         "use 16")
     ap.add_argument("--decode-only", action="store_true",
                     help="the step is the decode call alone (no kv_write)")
     ap.add_argument("--separate-write", action="store_true",
@@ -197,13 +200,17 @@ def _sharing_workload(name, model_block_manager):
     return wl, np.asarray(pairs, np.int32).reshape(-1, 2)
 
 
-def build_workload(name, model_block_manager=False):
+def build_workload(name, model_block_manager=False, block_size=16):
     """Return (Workload, cow_pairs int32 [P, 2]).  The fork workload's tables come from a
     block manager: the product's C++ one, or the oracle's Python model for the CPU arm."""
     from paged_kv_cache_392_b200 import workloads as W
+    if block_size != 16 and name not in ("opt13b", "gqa", "long"):
+        raise SystemExit("--block-size 32 applies to the opt13b, gqa and long workloads")
     if name in ("beam", "prefix"):
         return _sharing_workload(name, model_block_manager)
     if name != "fork":
+        if block_size != 16:
+            return W.CONFIGS[name](block_size=block_size), np.zeros((0, 2), np.int32)
         return W.CONFIGS[name](), np.zeros((0, 2), np.int32)
     f = W.FORK
     NB = W.fork_pool_blocks()
@@ -274,7 +281,8 @@ def contiguous_placement(wl):
     """Re-place every sequence's blocks back to back in pool order (block j of sequence s at
     pool block off_s + j): the layout a contiguous cache would have, read through the same
     block tables by the same kernel."""
-    nblk = (wl.context_lens.astype(np.int64) + 15) // 16
+    Bs = wl.block_size
+    nblk = (wl.context_lens.astype(np.int64) + Bs - 1) // Bs
     bt = np.full_like(wl.block_tables, -1)
     off = 0
     for s_, n in enumerate(nblk):
@@ -282,7 +290,7 @@ def contiguous_placement(wl):
         off += n
     wl.block_tables = bt
     pos = wl.context_lens.astype(np.int64) - 1
-    wl.slot_mapping = bt[np.arange(wl.num_seqs), pos // 16].astype(np.int64) * 16 + pos % 16
+    wl.slot_mapping = bt[np.arange(wl.num_seqs), pos // Bs].astype(np.int64) * Bs + pos % Bs
     wl.extra["placement"] = "contiguous"
 
 
@@ -294,12 +302,13 @@ def algorithmic_bytes(wl, pairs, split_rows=0, kv_es=None):
     S, Hq, Hkv, D = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim
     kv = int(wl.context_lens.astype(np.int64).sum()) * Hkv * D * kv_es * 2  # K and V once
     qo = S * Hq * D * es * 2                              # q read + out written
-    tables = int(((wl.context_lens + 15) // 16).sum()) * 4 + S * 4
+    Bs = wl.block_size
+    tables = int(((wl.context_lens + Bs - 1) // Bs).sum()) * 4 + S * 4
     ws = 0
     if split_rows:                                        # partials written + read
         ws = split_rows * (D + 2) * 4 * 2
     write = S * Hkv * D * (es + kv_es) * 2 + S * 8        # kv_write: read new + write pool
-    copy = len(pairs) * Hkv * 16 * D * kv_es * 2 * 2      # each pair: read + write K and V
+    copy = len(pairs) * Hkv * Bs * D * kv_es * 2 * 2      # each pair: read + write K and V
     return {"kv": kv, "decode": kv + qo + tables + ws, "kv_write": write, "kv_copy": copy,
             "step": kv + qo + tables + ws + write + copy}
 
@@ -315,15 +324,16 @@ def split_rows(wl, partition_tokens):
 def kv_utilisation(wl):
     """Fraction of the allocated KV slots that hold a token, from the block tables: every
     distinct physical block counts 16 slots once, filled as far as the furthest sequence that
-    maps it has written.  Without sharing this is sum(L) / (16 * sum(ceil(L / 16))); the
+    maps it has written.  Without sharing this is sum(L) / (B * sum(ceil(L / B))); the
     only waste is each sequence's partly filled last block."""
+    Bs = getattr(wl, "block_size", 16)
     fill = {}
     for s_, L in enumerate(wl.context_lens.astype(np.int64)):
-        nb = -(-int(L) // 16)
+        nb = -(-int(L) // Bs)
         for j in range(nb):
             b = int(wl.block_tables[s_, j])
-            fill[b] = max(fill.get(b, 0), min(16, int(L) - 16 * j))
-    slots = 16 * len(fill)
+            fill[b] = max(fill.get(b, 0), min(Bs, int(L) - Bs * j))
+    slots = Bs * len(fill)
     return {"tokens_in_blocks": int(sum(fill.values())), "slots_allocated": slots,
             "frac": round(sum(fill.values()) / slots, 4) if slots else None,
             "pages_figure": "about 96 % with 16-token blocks (vs 20-38 % for contiguous "
@@ -333,7 +343,7 @@ def kv_utilisation(wl):
 def uses_l2_flush(args, wl, nbytes, fp8):
     """Flush L2 between steps when the bytes a step really reads (shared blocks once) would
     fit in it twice over; otherwise the working set itself keeps L2 from carrying over."""
-    uniq_kv = (wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim *
+    uniq_kv = (wl.extra["unique_blocks"] * wl.num_kv_heads * wl.block_size * wl.head_dim *
                (1 if fp8 else wl.elem_size) * 2 if "unique_blocks" in wl.extra
                else nbytes["kv"])
     return bool(args.l2_flush or uniq_kv < 2 * L2_BYTES)
@@ -348,7 +358,7 @@ def step_config(args, wl, npairs, pt_run, nbytes, flush, fp8):
         "name": args.workload,
         "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
         "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
-        "block_size": 16, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
+        "block_size": wl.block_size, "kv_dtype": "fp8-e4m3" if fp8 else wl.dtype,
         "context_tokens": int(wl.context_lens.sum()),
         "partition_tokens": pt_run, "cow_pairs_per_step": npairs,
         "kv_bytes_per_step": nbytes["kv"], "step_bytes": nbytes["step"],
@@ -364,7 +374,7 @@ def step_config(args, wl, npairs, pt_run, nbytes, flush, fp8):
     }
     if args.layout == "contiguous":
         cfg["layout"] = ("contiguous [S][H_kv][Lmax][D] cache, Lmax = %d, no block table"
-                         % (wl.max_blocks_per_seq * 16))
+                         % (wl.max_blocks_per_seq * wl.block_size))
     return cfg
 
 
@@ -552,12 +562,12 @@ def time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ks
         used[wl.block_tables[wl.block_tables >= 0]] = True
         free = np.flatnonzero(~used)
         n = min(wl.num_seqs, len(free))
-        last = (wl.context_lens.astype(np.int64) - 1) // 16
+        last = (wl.context_lens.astype(np.int64) - 1) // wl.block_size
         src = wl.block_tables[np.arange(n), last[:n]]
         cp = np.stack([src, free[:n]], 1).astype(np.int32)
         source = "one per sequence: its last block into a block no table maps"
     cp_d = torch.from_numpy(cp).to(device)
-    copy_bytes = len(cp) * wl.num_kv_heads * 16 * wl.head_dim * kv_es * 2 * 2
+    copy_bytes = len(cp) * wl.num_kv_heads * wl.block_size * wl.head_dim * kv_es * 2 * 2
 
     def write():
         if fp8:
@@ -637,7 +647,7 @@ def run_pkv(args):
     torch.cuda.set_device(device)
     dist = init_dist(world)
 
-    wl, pairs = build_workload(args.workload)
+    wl, pairs = build_workload(args.workload, block_size=args.block_size)
     if args.contiguous:
         if args.workload in ("fork", "beam", "prefix"):
             raise SystemExit("--contiguous does not apply to the sharing workloads")
@@ -674,17 +684,18 @@ def run_pkv(args):
     fused = not args.separate_write and not decode_only
     kc = vc = None
     if contig:      # the same tokens in a [S][H_kv][Lmax][D] reservation per sequence
-        lmax = wl.max_blocks_per_seq * 16
+        Bs = wl.block_size
+        lmax = wl.max_blocks_per_seq * Bs
         kc = torch.zeros((wl.num_seqs, wl.num_kv_heads, lmax, wl.head_dim), dtype=kp.dtype,
                          device=device)
         vc = torch.zeros_like(kc)
         for s_ in range(wl.num_seqs):
             L = int(wl.context_lens[s_])
             t = torch.arange(L, device=device)
-            blk = bt[s_].long()[t // 16]
-            kc[s_, :, :L] = kp[blk, :, t % 16].permute(1, 0, 2)
-            vc[s_, :, :L] = vp[blk, :, t % 16].permute(1, 0, 2)
-        nbytes["decode"] -= int(((wl.context_lens + 15) // 16).sum()) * 4 + wl.num_seqs * 4
+            blk = bt[s_].long()[t // Bs]
+            kc[s_, :, :L] = kp[blk, :, t % Bs].permute(1, 0, 2)
+            vc[s_, :, :L] = vp[blk, :, t % Bs].permute(1, 0, 2)
+        nbytes["decode"] -= int(((wl.context_lens + Bs - 1) // Bs).sum()) * 4 + wl.num_seqs * 4
         nbytes["step"] = nbytes["decode"]
 
     def write(kn_, vn_, slots_):
@@ -1007,7 +1018,7 @@ def run_pkv(args):
             "clocks": sampler.summary(),
         }
         if "unique_blocks" in wl.extra:
-            uniq = wl.extra["unique_blocks"] * wl.num_kv_heads * 16 * wl.head_dim * \
+            uniq = wl.extra["unique_blocks"] * wl.num_kv_heads * wl.block_size * wl.head_dim * \
                 wl.elem_size * 2
             result["config"]["unique_kv_bytes"] = uniq
             result["unique_kv_gbs"] = round(world * uniq / (step_ms * 1e-3) / 1e9, 2)
@@ -1101,7 +1112,8 @@ def run_reference(args):
     import oracle
     import torch
     from paged_kv_cache_392_b200 import workloads as W
-    wl, pairs = build_workload(args.workload, model_block_manager=True)
+    wl, pairs = build_workload(args.workload, model_block_manager=True,
+                               block_size=args.block_size)
     if args.contiguous:
         contiguous_placement(wl)
     pt = args.partition_tokens if args.partition_tokens is not None else wl.partition_tokens

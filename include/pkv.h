@@ -5,9 +5,9 @@
  * Serving with PagedAttention" (sections "How PagedAttention Works" and "Advanced
  * Capabilities: Memory Sharing with Copy-on-Write") and "vLLM and PagedAttention: How Ideas
  * from Operating Systems Accelerated LLM Inference": the KV cache is a pool of fixed-size
- * physical blocks of 16 tokens, each sequence reaches its tokens through a block table, a
- * custom kernel gathers the scattered blocks to compute attention, and shared blocks are
- * copied before a sequence writes into them.
+ * physical blocks of 16 (or 32) tokens, each sequence reaches its tokens through a block
+ * table, a custom kernel gathers the scattered blocks to compute attention, and shared blocks
+ * are copied before a sequence writes into them.
  *
  * Conventions (every function):
  *   - Returns pkv_status; PKV_OK is 0.  On failure pkv_last_error() (per calling thread)
@@ -18,9 +18,10 @@
  *     are asynchronous; the calls return once the kernels are queued.
  *   - dtype is one of pkv_dtype; q, out, the pools and the new K/V all use the same dtype.
  *   - Pool layout: k_pool and v_pool are row-major [num_blocks][num_kv_heads][block_size]
- *     [head_dim], so one (block, kv head) is a contiguous block_size*head_dim run.
- *     Token t of sequence s is at block block_tables[s*max_blocks_per_seq + t/16], offset
- *     t%16.  A slot number names (block, offset) as block*16 + offset.
+ *     [head_dim], so one (block, kv head) is a contiguous block_size*head_dim run.  With
+ *     B = block_size (16 or 32), token t of sequence s is at block
+ *     block_tables[s*max_blocks_per_seq + t/B], offset t%B.  A slot number names (block,
+ *     offset) as block*B + offset.
  *   - Device-side checks: values only the GPU sees (context lengths, table entries, slots,
  *     block ids) are range-checked by the kernels before any access.  A bad value is skipped
  *     (never dereferenced) and sets a bit in the device fault word that
@@ -71,7 +72,7 @@ typedef struct pkv_attn_desc {
     int32_t num_kv_heads;        /* H_kv; H_q % H_kv == 0, query head h reads kv head   */
                                  /* h / (H_q / H_kv)                                    */
     int32_t head_dim;            /* D: 64 or 128                                        */
-    int32_t block_size;          /* tokens per block: 16                                */
+    int32_t block_size;          /* tokens per block B: 16 or 32                        */
     int32_t num_blocks;          /* NB, physical blocks in each pool                    */
     int32_t max_blocks_per_seq;  /* row stride of block_tables                          */
     int32_t dtype;               /* pkv_dtype                                           */
@@ -101,10 +102,10 @@ size_t pkv_attn_workspace_bytes(const pkv_attn_desc *desc);
  *     out[s,h,:] = sum_t softmax(x)_t * V_t
  * accumulated in fp32 and rounded once to dtype.
  *   q            [S, H_q, D] dtype
- *   k_pool/v_pool [NB, H_kv, 16, D] dtype, 16-byte aligned
+ *   k_pool/v_pool [NB, H_kv, B, D] dtype, 16-byte aligned
  *   block_tables [S, max_blocks_per_seq] int32; only the first ceil(L/16) entries of a row
  *                are read
- *   context_lens [S] int32, each in [1, max_blocks_per_seq*16] (checked on the device)
+ *   context_lens [S] int32, each in [1, max_blocks_per_seq*B] (checked on the device)
  *   out          [S, H_q, D] dtype
  *   workspace    at least pkv_attn_workspace_bytes(desc) bytes, 256-byte aligned (may be
  *                NULL when that is 0); overwritten; calls that share it must not overlap
@@ -123,7 +124,7 @@ pkv_status paged_attn_decode(const pkv_attn_desc *desc, const void *q, const voi
  *     k_pool[slot/16, h, slot%16, :] = k_new[t, h, :]   (and the same for V)
  * bytes copied unchanged.  slot_mapping[t] == -1 skips token t.
  *   k_new/v_new  [num_tokens, H_kv, D] dtype
- *   slot_mapping [num_tokens] int64, distinct values in [0, NB*16) or -1
+ *   slot_mapping [num_tokens] int64, distinct values in [0, NB*B) or -1
  * Checked on the device: a slot outside the pool is skipped (PKV_FAULT_BAD_SLOT); a slot
  * that two or more tokens of the call name is skipped for all of them
  * (PKV_FAULT_DUPLICATE), so the pools never depend on which write lands last.  The check
@@ -146,7 +147,7 @@ pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_
  * bit for bit, under these conditions:
  *   - token s of k_new / v_new ([S, H_kv, D] dtype, 16-byte aligned) belongs to sequence s,
  *     and slot_mapping[s] (int64 [S], 8-byte aligned) is -1 (no write) or the slot of
- *     position context_lens[s]-1, i.e. block_tables[s][(L-1)/16]*16 + (L-1)%16;
+ *     position context_lens[s]-1, i.e. block_tables[s][(L-1)/B]*B + (L-1)%B;
  *   - the block holding that slot is read by no other sequence of the batch (copy-on-write
  *     of shared blocks, kv_copy_blocks, must already have run; the block manager's
  *     append_slot(s) guarantees this).
@@ -168,8 +169,8 @@ pkv_status kv_write_and_decode(const pkv_attn_desc *desc, const void *q, const v
  * what paged_attn_decode computes (same kernel body, same partitions and rounding), with
  * token t of sequence s and kv head h at row t of a reservation of Lmax token rows:
  *   k_cache/v_cache [S, H_kv, Lmax, D] dtype (f16 or bf16), 16-byte aligned, where
- *                   Lmax = desc->max_blocks_per_seq * 16 (rows past context_lens[s] are
- *                   never used)
+ *                   Lmax = desc->max_blocks_per_seq * desc->block_size (rows past
+ *                   context_lens[s] are never used)
  *   context_lens    [S] int32, each in [1, Lmax] (checked on the device)
  * q, out, scale, the workspace (pkv_attn_workspace_bytes(desc)) and the errors are as
  * paged_attn_decode's; desc->num_blocks is not used.  S * H_kv * Lmax must stay below 2^31.
@@ -200,7 +201,7 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
  * Swap whole blocks between the device pools and a host pool ("vLLM and PagedAttention: How
  * Ideas from Operating Systems Accelerated LLM Inference": when memory runs short, whole
  * sequences are evicted by swapping them to CPU memory).  host_k / host_v are pinned host
- * buffers of num_host_blocks blocks, [num_host_blocks][H_kv][16][D] dtype each, allocated
+ * buffers of num_host_blocks blocks, [num_host_blocks][H_kv][B][D] dtype each, allocated
  * so the device can reach them (cudaHostAlloc / cudaMallocHost, or torch pin_memory); other
  * host memory is rejected with PKV_ERR_INVALID before any launch.  pairs is device int32
  * [num_pairs][2]:
@@ -227,8 +228,9 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  *     and means code * scale.  A head whose K or V scale is not finite and > 0 sets
  *     PKV_FAULT_BAD_SCALE: the writes skip that head's values and the decode's output for
  *     its query heads is unspecified;
- *   - k_pool: [NB][H_kv][16][D] bytes;  v_pool: [NB][H_kv][D][16] bytes, transposed, where
- *     slot p of a row holds token 2*(p>>2) + (p&1) + 8*((p>>1)&1) of the block.
+ *   - k_pool: [NB][H_kv][B][D] bytes;  v_pool: [NB][H_kv][B/16][D][16] bytes: each
+ *     16-token half of a block transposed, slot p of a row holding token
+ *     2*(p>>2) + (p&1) + 8*((p>>1)&1) of the half (for B = 16 this is [NB][H_kv][D][16]).
  * Only head_dim 128 is built.  Pools are 16-byte aligned.  kv_copy_blocks and kv_swap_* move
  * these blocks with desc->dtype = PKV_FP8_E4M3.
  *
@@ -333,13 +335,13 @@ pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream);
 typedef struct pkv_bm pkv_bm;
 
 /* initial_free_order: host [num_blocks] permutation of 0..num_blocks-1, or NULL for
- * ascending order.  block_size must be 16. */
+ * ascending order.  block_size is 16 or 32. */
 pkv_status pkv_bm_create(int32_t num_blocks, int32_t block_size,
                          const int32_t *initial_free_order, pkv_bm **out);
 void pkv_bm_destroy(pkv_bm *bm);
 
-/* Register sequence seq holding num_tokens tokens (a prompt): ceil(num_tokens/16) fresh
- * blocks, all or nothing. */
+/* Register sequence seq holding num_tokens tokens (a prompt): ceil(num_tokens/block_size)
+ * fresh blocks, all or nothing. */
 pkv_status pkv_bm_add_seq(pkv_bm *bm, int64_t seq, int32_t num_tokens);
 
 /* Give the next token of seq a slot.  If the token opens a new block, a fresh block is

@@ -167,7 +167,7 @@ def _pool_desc(k_pool, v_pool, num_seqs=0, num_q_heads=1, max_blocks_per_seq=1,
     _dev(k_pool, "k_pool")
     _dev(v_pool, "v_pool", k_pool.dtype)
     if k_pool.dim() != 4 or v_pool.shape != k_pool.shape:
-        raise ValueError("pools must both be [num_blocks, num_kv_heads, 16, head_dim]")
+        raise ValueError("pools must both be [num_blocks, num_kv_heads, block_size, head_dim]")
     NB, Hkv, B, D = k_pool.shape
     if k_pool.dtype not in DTYPE_CODE:
         raise TypeError("unsupported pool dtype %s" % k_pool.dtype)
@@ -342,7 +342,7 @@ def _block_pools_desc(k_pool, v_pool):
     [NB, H_kv, D, 16]; a block's bytes are moved the same way)."""
     if k_pool.dtype == torch.uint8:
         NB, Hkv, Bs, D = _fp8_pools(k_pool, v_pool)
-        return make_desc(0, Hkv, Hkv, D, NB, 1, PKV_FP8_E4M3)
+        return make_desc(0, Hkv, Hkv, D, NB, 1, PKV_FP8_E4M3, 0, Bs)
     return _pool_desc(k_pool, v_pool)
 
 
@@ -391,12 +391,16 @@ def kv_swap_in(pairs, host_k, host_v, k_pool, v_pool, stream=None):
 
 
 def _fp8_pools(k_pool, v_pool):
-    """FP8 pools: K [NB, H_kv, 16, D] and V [NB, H_kv, D, 16], uint8 E4M3 codes."""
+    """FP8 pools, uint8 E4M3 codes: K [NB, H_kv, B, D] and V [NB, H_kv, B/16, D, 16] (each
+    16-token half of a block transposed), which for B = 16 may also be [NB, H_kv, D, 16]."""
     _dev(k_pool, "k_pool", torch.uint8)
     _dev(v_pool, "v_pool", torch.uint8)
-    if k_pool.dim() != 4 or v_pool.shape != (k_pool.shape[0], k_pool.shape[1],
-                                             k_pool.shape[3], k_pool.shape[2]):
-        raise ValueError("FP8 pools: K [NB, H_kv, 16, D], V [NB, H_kv, D, 16]")
+    if k_pool.dim() != 4:
+        raise ValueError("FP8 K pool: [NB, H_kv, B, D]")
+    NB, Hkv, Bs, D = k_pool.shape
+    if v_pool.shape != (NB, Hkv, Bs // 16, D, 16) and not (
+            Bs == 16 and v_pool.shape == (NB, Hkv, D, 16)):
+        raise ValueError("FP8 V pool: [NB, H_kv, B/16, D, 16] (or [NB, H_kv, D, 16] for B 16)")
     return k_pool.shape
 
 

@@ -41,7 +41,10 @@ namespace pkv {
 #endif
 constexpr int kDefaultPartitionTokens = 512;
 
-constexpr int kBlock = 16;                       // tokens per KV block
+// Tokens per KV sub-block: the unit every kernel stages and multiplies (one TMA box, one MMA
+// tile).  A physical block holds 16 or 32 tokens (1 << DecodeParams::bshift): sub-block j of
+// a sequence is rows 16 * (j mod (B / 16)) .. of physical block block_tables[s][j / (B / 16)].
+constexpr int kBlock = 16;
 // Lazy online-softmax rescale threshold (base-2 logit units): a running max moves only when
 // a block's max exceeds it by more than this, so exponents stay <= 2^8.
 #ifndef PKV_LAZY_RESCALE
@@ -90,7 +93,16 @@ struct DecodeParams {
     // contiguous cache (attn_decode_contiguous): token rows per (sequence, kv head); 0 for
     // the paged pools
     int32_t Lmax = 0;
+    // log2 of the tokens per physical block (4: 16-token blocks, 5: 32-token blocks)
+    int32_t bshift = 4;
 };
+
+// Table entry of sub-block j (of kBlock tokens) and the sub-block's first row within its
+// physical block: sub-block j lies in table entry j >> (bshift - 4), at row 16 * (j & ...).
+__device__ __forceinline__ int sub_to_entry(int j, int bshift) { return j >> (bshift - 4); }
+__device__ __forceinline__ int sub_row(int j, int bshift) {
+    return (j & ((1 << (bshift - 4)) - 1)) * kBlock;
+}
 
 // Fused kv_write, called by the one warp per (sequence, kv head) that will copy the block
 // holding position L-1.  The warp stores the newest token's K and V rows of kv head hk into
@@ -102,12 +114,12 @@ __device__ __forceinline__ void write_newest_token(const DecodeParams &p, int s,
                                                    int lane) {
     const int64_t slot = p.slot_mapping[s];
     if (slot != -1) {
-        const int32_t blk = p.block_tables[(size_t)s * p.maxB + (L - 1) / kBlock];
-        const int off = (L - 1) % kBlock;
-        if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
+        const int32_t blk = p.block_tables[(size_t)s * p.maxB + ((L - 1) >> p.bshift)];
+        const int off = (L - 1) & ((1 << p.bshift) - 1);
+        if ((unsigned)blk < (unsigned)p.NB && slot == ((int64_t)blk << p.bshift) + off) {
             constexpr int VPR = D * (int)sizeof(T) / 16;  // 16-byte vectors per row
             const size_t src = ((size_t)s * p.Hkv + hk) * VPR;
-            const size_t dst = (((size_t)blk * p.Hkv + hk) * kBlock + off) * VPR;
+            const size_t dst = ((((size_t)blk * p.Hkv + hk) << p.bshift) + off) * VPR;
             // the pools are written only here; the decode itself reads them
             uint4 *kp = static_cast<uint4 *>(const_cast<void *>(p.k_pool));
             uint4 *vp = static_cast<uint4 *>(const_cast<void *>(p.v_pool));
@@ -296,7 +308,7 @@ paged_attn_decode_kernel(const DecodeParams p) {
     const int s = rest / p.Hkv;
 
     const int L = p.context_lens[s];
-    if (L < 1 || L > p.maxB * kBlock) {
+    if (L < 1 || L > (p.maxB << p.bshift)) {
         if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
@@ -328,28 +340,31 @@ paged_attn_decode_kernel(const DecodeParams p) {
     if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
         write_newest_token<T, D>(p, s, hk, L, lane);
 
-    const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const int32_t *btab = p.block_tables + (size_t)s * p.maxB;
+    const int j1 = j0 + warp;  // this warp's first sub-block
     const char *kbase = static_cast<const char *>(p.k_pool);
     const char *vbase = static_cast<const char *>(p.v_pool);
     const uint64_t policy = l2_evict_first_policy();
 
-    // Block-table entries of this warp's blocks, 32 at a time (lane i holds block i).
+    // Block-table entries of this warp's sub-blocks, 32 at a time (lane i holds sub-block i).
     int tab_chunk = 0;
-    int32_t tab = lane < nbw ? btrow[(size_t)W * lane] : 0;
+    int32_t tab = lane < nbw ? btab[sub_to_entry(j1 + W * lane, p.bshift)] : 0;
 
-    // Issue block i of this warp into stage i % NSW (all lanes call; lane 0 issues).
+    // Issue sub-block i of this warp into stage i % NSW (all lanes call; lane 0 issues).
     auto issue = [&](int i) {
         if ((i >> 5) != tab_chunk) {
             tab_chunk = i >> 5;
             const int li = (tab_chunk << 5) + lane;
-            tab = li < nbw ? btrow[(size_t)W * li] : 0;
+            tab = li < nbw ? btab[sub_to_entry(j1 + W * li, p.bshift)] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
         if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * 2 * CHUNK;
             if ((unsigned)phys < (unsigned)p.NB) {
-                const size_t off = ((size_t)phys * p.Hkv + hk) * (size_t)CHUNK;
+                const size_t row = (((size_t)phys * p.Hkv + hk) << p.bshift) +
+                                   (size_t)sub_row(j1 + W * i, p.bshift);
+                const size_t off = row * (size_t)(CHUNK / kBlock);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, 2 * CHUNK);
                 bulk_g2s(dst, kbase + off, CHUNK, bar, policy);
@@ -566,7 +581,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     if (row >= p.S * p.Hq) return;
     const int s = row / p.Hq;
     const int L = p.context_lens[s];
-    if (L < 1 || L > p.maxB * kBlock) return;
+    if (L < 1 || L > (p.maxB << p.bshift)) return;
     const int nblk = (L + kBlock - 1) / kBlock;
     const int np = (nblk + p.part_blocks - 1) / p.part_blocks;
     if (np <= 1) return;

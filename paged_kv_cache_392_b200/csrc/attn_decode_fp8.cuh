@@ -6,10 +6,11 @@
 //   * each KV head has one fp32 scale for K and one for V; element x is stored as the E4M3
 //     code of x / scale (fp32 division, round to nearest even, saturating to +-448) and
 //     means code * scale;
-//   * K blocks: [block][kv head][16 tokens][D] bytes (as the 16-bit pools);
-//   * V blocks: [block][kv head][D][16 slots] bytes -- transposed, and slot p of a row holds
-//     token 2*(p>>2) + (p&1) + 8*((p>>1)&1) (v_slot_of_token below is the inverse), so that
-//     the 4 bytes an ldmatrix lane reads from a row are the token pairs the P.V tile wants.
+//   * K blocks: [block][kv head][B tokens][D] bytes (as the 16-bit pools), B = 16 or 32;
+//   * V blocks: [block][kv head][B/16][D][16 slots] bytes -- each 16-token half of a block
+//     transposed, and slot p of a row holds token 2*(p>>2) + (p&1) + 8*((p>>1)&1) of the
+//     half (v_slot_of_token below is the inverse), so that the 4 bytes an ldmatrix lane
+//     reads from a row are the token pairs the P.V tile wants.
 // Decode: q.K^T runs on m16n8k32 E4M3 tensor-core tiles straight from the K codes, with each
 // query row prescaled by a power of two and split into two E4M3 terms (hi + residual, about
 // bfloat16 precision; with at most four query heads per kv head both terms ride in one MMA
@@ -123,24 +124,27 @@ __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp
     const DecodeParams &p = fp.base;
     const int64_t slot = p.slot_mapping[s];
     if (slot != -1) {
-        const int32_t blk = p.block_tables[(size_t)s * p.maxB + (L - 1) / kBlock];
-        const int off = (L - 1) % kBlock;
+        const int32_t blk = p.block_tables[(size_t)s * p.maxB + ((L - 1) >> p.bshift)];
+        const int off = (L - 1) & ((1 << p.bshift) - 1);
         const float ksc = fp.k_scale[hk], vsc = fp.v_scale[hk];
         if (!scale_ok(ksc) || !scale_ok(vsc)) {
             if (lane == 0) atomicOr(&g_faults, kFaultBadScale);
-        } else if ((unsigned)blk < (unsigned)p.NB && slot == (int64_t)blk * kBlock + off) {
+        } else if ((unsigned)blk < (unsigned)p.NB && slot == ((int64_t)blk << p.bshift) + off) {
             const int64_t src = ((int64_t)s * p.Hkv + hk) * D;
             const int64_t hb = (int64_t)blk * p.Hkv + hk;
-            const int vs = v_slot_of_token(off);
+            // the 16-token half of the block that holds the token, and its V^T slot
+            const int64_t vh = (hb << (p.bshift - 4)) + (off >> 4);
+            const int vs = v_slot_of_token(off & 15);
             // the pools are written only here; the decode itself reads them
             uint8_t *kp = static_cast<uint8_t *>(const_cast<void *>(p.k_pool));
             uint8_t *vp = static_cast<uint8_t *>(const_cast<void *>(p.v_pool));
             for (int d = 2 * lane; d < D; d += 64) {
                 const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src + d, ksc);
                 const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src + d, vsc);
-                *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + (hb * kBlock + off) * D + d) = kc;
-                vp[(hb * D + d) * kBlock + vs] = static_cast<uint8_t>(vc & 0xffu);
-                vp[(hb * D + d + 1) * kBlock + vs] = static_cast<uint8_t>(vc >> 8);
+                *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + ((hb << p.bshift) + off) * D +
+                                                          d) = kc;
+                vp[(vh * D + d) * kBlock + vs] = static_cast<uint8_t>(vc & 0xffu);
+                vp[(vh * D + d + 1) * kBlock + vs] = static_cast<uint8_t>(vc >> 8);
             }
             fence_proxy_async_global();
         } else if (lane == 0) {
@@ -201,7 +205,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     const int s = rest / p.Hkv;
 
     const int L = p.context_lens[s];
-    if (L < 1 || L > p.maxB * kBlock) {
+    if (L < 1 || L > (p.maxB << p.bshift)) {
         if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
@@ -232,29 +236,34 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
         write_newest_token_fp8<T>(fp, s, hk, L, lane);
 
-    const int32_t *btrow = p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const int32_t *btab = p.block_tables + (size_t)s * p.maxB;
+    const int j1 = j0 + warp;  // this warp's first sub-block
     const char *vbase = static_cast<const char *>(p.v_pool);
     const uint64_t policy = l2_evict_first_policy();
     int tab_chunk = 0;
-    int32_t tab = lane < nbw ? btrow[(size_t)W * lane] : 0;
+    int32_t tab = lane < nbw ? btab[sub_to_entry(j1 + W * lane, p.bshift)] : 0;
 
     auto issue = [&](int i) {
         if ((i >> 5) != tab_chunk) {
             tab_chunk = i >> 5;
             const int li = (tab_chunk << 5) + lane;
-            tab = li < nbw ? btrow[(size_t)W * li] : 0;
+            tab = li < nbw ? btab[sub_to_entry(j1 + W * li, p.bshift)] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
         if (lane == 0 && !withheld_for_test(i, warp)) {
             uint64_t *bar = &bars[i % NSW];
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
             if ((unsigned)phys < (unsigned)p.NB) {
-                const int32_t row = (phys * p.Hkv + hk) * kBlock;
+                const int jb = j1 + W * i;
+                const int32_t row = ((phys * p.Hkv + hk) << p.bshift) + sub_row(jb, p.bshift);
+                // V^T of the sub-block: the 16-token half (jb's position in the block) of
+                // the block's [B/16][D][16] bytes
+                const size_t vhalf = ((size_t)(phys * p.Hkv + hk) << (p.bshift - 4)) +
+                                     (size_t)(sub_row(jb, p.bshift) / kBlock);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, 2 * CHUNK);
                 tma_load_2d(dst, &tmk, 0, row, bar, policy);
-                bulk_g2s(dst + CHUNK, vbase + (size_t)(phys * p.Hkv + hk) * CHUNK, CHUNK, bar,
-                         policy);
+                bulk_g2s(dst + CHUNK, vbase + vhalf * CHUNK, CHUNK, bar, policy);
             } else {
                 atomicOr(&g_faults, kFaultBadBlock);
                 mbar_arrive(bar);
@@ -574,9 +583,10 @@ struct KvWriteFp8Params {
     const int64_t *slot_mapping;
     const float *k_scale;
     const float *v_scale;
-    uint8_t *k_pool;    // [NB][H_kv][16][D]
-    uint8_t *v_pool;    // [NB][H_kv][D][16] (slot order v_slot_of_token)
+    uint8_t *k_pool;    // [NB][H_kv][B][D]
+    uint8_t *v_pool;    // [NB][H_kv][B/16][D][16] (slot order v_slot_of_token)
     int32_t T, Hkv, NB, D;
+    int32_t bshift;     // log2 B (4 or 5)
 };
 
 
@@ -599,7 +609,7 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_fp8_kernel(const KvWri
         const int h = hd / (p.D / 2), d = 2 * (hd % (p.D / 2));
         const int64_t slot = ts.slot[tl];
         if (slot == -1) continue;
-        if (slot < 0 || slot >= (int64_t)p.NB * 16) {
+        if (slot < 0 || slot >= ((int64_t)p.NB << p.bshift)) {
             if (hd == 0) atomicOr(&g_faults, kFaultBadSlot);
             continue;
         }
@@ -612,16 +622,18 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_fp8_kernel(const KvWri
             if (d == 0) atomicOr(&g_faults, kFaultBadScale);
             continue;
         }
-        const int64_t blk = slot >> 4;
-        const int off = (int)(slot & 15);
+        const int64_t blk = slot >> p.bshift;
+        const int off = (int)(slot & ((1 << p.bshift) - 1));
         const int64_t src = ((t0 + tl) * p.Hkv + h) * p.D + d;
         const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src, ksc);
         const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src, vsc);
         const int64_t hb = blk * p.Hkv + h;
-        *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + (hb * 16 + off) * p.D + d) = kc;
-        const int sp = v_slot_of_token(off);
-        p.v_pool[(hb * p.D + d) * 16 + sp] = static_cast<uint8_t>(vc & 0xffu);
-        p.v_pool[(hb * p.D + d + 1) * 16 + sp] = static_cast<uint8_t>(vc >> 8);
+        *reinterpret_cast<__nv_fp8x2_storage_t *>(p.k_pool + ((hb << p.bshift) + off) * p.D +
+                                                  d) = kc;
+        const int64_t vh = (hb << (p.bshift - 4)) + (off >> 4);  // the token's 16-token half
+        const int sp = v_slot_of_token(off & 15);
+        p.v_pool[(vh * p.D + d) * 16 + sp] = static_cast<uint8_t>(vc & 0xffu);
+        p.v_pool[(vh * p.D + d + 1) * 16 + sp] = static_cast<uint8_t>(vc >> 8);
     }
 }
 

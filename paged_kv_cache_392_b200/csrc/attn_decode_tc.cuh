@@ -82,7 +82,7 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
     const int s = rest / p.Hkv;
 
     const int L = p.context_lens[s];
-    if (L < 1 || L > p.maxB * kBlock) {
+    if (L < 1 || L > (p.maxB << p.bshift)) {
         if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
@@ -116,10 +116,11 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
     if (!kContig && p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
         write_newest_token<T, D>(p, s, hk, L, lane);
 
-    const int32_t *btrow = kContig ? nullptr : p.block_tables + (size_t)s * p.maxB + j0 + warp;
+    const int32_t *btab = kContig ? nullptr : p.block_tables + (size_t)s * p.maxB;
+    const int j1 = j0 + warp;  // this warp's first sub-block
     const uint64_t policy = l2_evict_first_policy();
     int tab_chunk = 0;
-    int32_t tab = !kContig && lane < nbw ? btrow[(size_t)W * lane] : 0;
+    int32_t tab = !kContig && lane < nbw ? btab[sub_to_entry(j1 + W * lane, p.bshift)] : 0;
     // contiguous cache: TMA row of this warp's first block
     const int32_t crow0 = kContig ? (s * p.Hkv + hk) * p.Lmax + (j0 + warp) * kBlock : 0;
 
@@ -130,7 +131,7 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
             if ((i >> 5) != tab_chunk) {
                 tab_chunk = i >> 5;
                 const int li = (tab_chunk << 5) + lane;
-                tab = li < nbw ? btrow[(size_t)W * li] : 0;
+                tab = li < nbw ? btab[sub_to_entry(j1 + W * li, p.bshift)] : 0;
             }
             phys = __shfl_sync(FULL, tab, i & 31);
         }
@@ -139,7 +140,8 @@ __device__ __forceinline__ void decode_tc_body(const CUtensorMap &tmk, const CUt
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
             if (kContig || (unsigned)phys < (unsigned)p.NB) {
                 const int32_t row = kContig ? crow0 + i * (W * kBlock)
-                                            : (phys * p.Hkv + hk) * kBlock;
+                                            : ((phys * p.Hkv + hk) << p.bshift) +
+                                                  sub_row(j1 + W * i, p.bshift);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, 2 * CHUNK);
 #pragma unroll

@@ -110,8 +110,8 @@ pkv_status pkv_bm_create(int32_t num_blocks, int32_t block_size,
     if (!out) return fail(PKV_ERR_INVALID, "pkv_bm_create: out is NULL");
     *out = nullptr;
     if (num_blocks < 0) return fail(PKV_ERR_INVALID, "pkv_bm_create: num_blocks < 0");
-    if (block_size != 16)
-        return fail(PKV_ERR_UNSUPPORTED, "pkv_bm_create: block_size %d (only 16)", block_size);
+    if (block_size != 16 && block_size != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "pkv_bm_create: block_size %d (16 or 32)", block_size);
     pkv_bm *bm = new (std::nothrow) pkv_bm;
     if (!bm) return fail(PKV_ERR_OOM, "pkv_bm_create: host allocation failed");
     bm->num_blocks = num_blocks;

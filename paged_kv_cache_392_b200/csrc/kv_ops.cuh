@@ -67,10 +67,11 @@ struct KvWriteParams {
     const uint4 *k_new;  // [T][H_kv][D] as 16-byte vectors
     const uint4 *v_new;
     const int64_t *slot_mapping;
-    uint4 *k_pool;       // [NB][H_kv][16][D]
+    uint4 *k_pool;       // [NB][H_kv][B][D]
     uint4 *v_pool;
     int32_t T, Hkv, NB;
     int32_t vpr;         // 16-byte vectors per row (D * elem_size / 16)
+    int32_t bshift;      // log2 B: tokens per block (16 or 32)
 };
 
 // grid.x = tile of kTileTokens tokens, grid.y = slice of the tile's vectors.  Within a tile
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(const KvWritePa
         const int64_t slot = ts.slot[tl];
         if (slot == -1) continue;
         const bool reporter = which == 0 && hc == 0;   // one report per token
-        if (slot < 0 || slot >= (int64_t)p.NB * 16) {
+        if (slot < 0 || slot >= ((int64_t)p.NB << p.bshift)) {
             if (reporter) atomicOr(&g_faults, kFaultBadSlot);
             continue;
         }
@@ -100,7 +101,8 @@ __global__ void __launch_bounds__(kWriteThreads) kv_write_kernel(const KvWritePa
             continue;
         }
         const int h = hc / p.vpr, c = hc % p.vpr;
-        const int64_t dst = (((slot >> 4) * p.Hkv + h) * 16 + (slot & 15)) * p.vpr + c;
+        const int64_t dst = ((((slot >> p.bshift) * p.Hkv + h) << p.bshift) +
+                             (slot & ((1 << p.bshift) - 1))) * p.vpr + c;
         const int64_t src = (t0 + tl) * per_tok + hc;
         if (which == 0)
             p.k_pool[dst] = p.k_new[src];

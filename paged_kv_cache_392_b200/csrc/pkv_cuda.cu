@@ -34,20 +34,27 @@ int elem_size(int32_t dtype) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// log2 of the tokens per physical block (16 or 32; checked by check_pool_desc).
+int32_t block_shift(const pkv_attn_desc *d) { return d->block_size == 32 ? 5 : 4; }
+
+// 16-token sub-blocks the longest admissible sequence spans.
+int64_t sub_blocks_per_seq(const pkv_attn_desc *d) {
+    return (int64_t)d->max_blocks_per_seq * (d->block_size / pkv::kBlock);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Checks shared by every entry point that touches the pools.
 pkv_status check_pool_desc(const pkv_attn_desc *d, const char *fn) {
     if (!d) return fail(PKV_ERR_INVALID, "%s: desc is NULL", fn);
     if (!elem_size(d->dtype)) return fail(PKV_ERR_INVALID, "%s: unknown dtype %d", fn, d->dtype);
-    if (d->block_size != pkv::kBlock)
-        return fail(PKV_ERR_UNSUPPORTED, "%s: block_size %d (only 16 is built)", fn,
-                    d->block_size);
+    if (d->block_size != 16 && d->block_size != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "%s: block_size %d (16 or 32)", fn, d->block_size);
     if (d->head_dim != 64 && d->head_dim != 128)
         return fail(PKV_ERR_UNSUPPORTED, "%s: head_dim %d (64 or 128)", fn, d->head_dim);
     if (d->num_kv_heads < 1) return fail(PKV_ERR_INVALID, "%s: num_kv_heads < 1", fn);
     if (d->num_blocks < 1) return fail(PKV_ERR_INVALID, "%s: num_blocks < 1", fn);
-    if ((int64_t)d->num_blocks * pkv::kBlock > INT64_MAX / 2)
+    if ((int64_t)d->num_blocks * d->block_size > INT64_MAX / 2)
         return fail(PKV_ERR_INVALID, "%s: num_blocks too large", fn);
     return PKV_OK;
 }
@@ -71,14 +78,14 @@ pkv_status check_attn_desc(const pkv_attn_desc *d, const char *fn, Split *sp) {
         return fail(PKV_ERR_UNSUPPORTED, "%s: query heads per kv head %d (1, 2, 4 or 8)", fn, g);
     if (d->dtype == PKV_F32 && d->head_dim == 128 && g == 8)
         return fail(PKV_ERR_UNSUPPORTED, "%s: fp32 with head_dim 128 and group 8", fn);
-    if (d->max_blocks_per_seq < 1 || d->max_blocks_per_seq > INT_MAX / pkv::kBlock)
+    if (d->max_blocks_per_seq < 1 || d->max_blocks_per_seq > INT_MAX / d->block_size)
         return fail(PKV_ERR_INVALID, "%s: max_blocks_per_seq %d", fn, d->max_blocks_per_seq);
     if (d->partition_tokens < 0 || d->partition_tokens % pkv::kBlock)
         return fail(PKV_ERR_INVALID, "%s: partition_tokens %d not a multiple of 16", fn,
                     d->partition_tokens);
     const int32_t pt = d->partition_tokens ? d->partition_tokens : kDefaultPartitionTokens;
-    sp->part_blocks = pt / pkv::kBlock;
-    sp->pmax = (d->max_blocks_per_seq + sp->part_blocks - 1) / sp->part_blocks;
+    sp->part_blocks = pt / pkv::kBlock;  // partitions count 16-token sub-blocks
+    sp->pmax = (sub_blocks_per_seq(d) + sp->part_blocks - 1) / sp->part_blocks;
     const int64_t grid = (int64_t)d->num_seqs * d->num_kv_heads * sp->pmax;
     if (grid > INT_MAX || (int64_t)d->num_seqs * d->num_q_heads > INT_MAX)
         return fail(PKV_ERR_INVALID, "%s: batch too large for one launch", fn);
@@ -175,7 +182,7 @@ pkv_status launch_decode_tc(const pkv::DecodeParams &prm, int32_t dtype, cudaStr
     pkv_status st = ensure_smem(kern, Cfg::SMEM, done, "paged_attn_decode");
     if (st) return st;
     const int64_t rows = kContig ? (int64_t)prm.S * prm.Hkv * prm.Lmax
-                                 : (int64_t)prm.NB * prm.Hkv * pkv::kBlock;
+                                 : ((int64_t)prm.NB * prm.Hkv) << prm.bshift;
     CUtensorMap tmk, tmv;
     st = kv_tensor_map(&tmk, prm.k_pool, dtype, D, rows, "paged_attn_decode");
     if (st) return st;
@@ -210,7 +217,7 @@ bool use_tc(const pkv_attn_desc *d) {
     return false;
 #else
     return d->dtype != PKV_F32 &&
-           (int64_t)d->num_blocks * d->num_kv_heads * pkv::kBlock < ((int64_t)1 << 31);
+           (int64_t)d->num_blocks * d->num_kv_heads * d->block_size < ((int64_t)1 << 31);
 #endif
 }
 
@@ -316,6 +323,7 @@ pkv_status decode_impl(const pkv_attn_desc *desc, const void *q, const void *k_n
     prm.part_blocks = sp.part_blocks;
     prm.pmax = sp.pmax;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.bshift = block_shift(desc);
     const int g = desc->num_q_heads / desc->num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (use_tc(desc)) {
@@ -396,6 +404,7 @@ pkv_status kv_write(const pkv_attn_desc *desc, const void *k_new, const void *v_
     prm.Hkv = desc->num_kv_heads;
     prm.NB = desc->num_blocks;
     prm.vpr = desc->head_dim * elem_size(desc->dtype) / 16;
+    prm.bshift = block_shift(desc);
     dim3 grid;
     st = write_grid(num_tokens, 2LL * prm.Hkv * prm.vpr, &grid, fn);
     if (st) return st;
@@ -421,7 +430,7 @@ pkv_status kv_copy_blocks(const pkv_attn_desc *desc, const int32_t *src_dst_pair
     prm.v_pool = static_cast<uint4 *>(v_pool);
     prm.P = num_pairs;
     prm.NB = desc->num_blocks;
-    prm.vpb = (int64_t)desc->num_kv_heads * pkv::kBlock * desc->head_dim *
+    prm.vpb = (int64_t)desc->num_kv_heads * desc->block_size * desc->head_dim *
               elem_size(desc->dtype) / 16;
     const int64_t slices = (prm.vpb + pkv::kCopyUnroll * 256 - 1) / (pkv::kCopyUnroll * 256);
     if (slices > 65535) return fail(PKV_ERR_UNSUPPORTED, "%s: block too large", fn);
@@ -440,7 +449,7 @@ pkv_status attn_decode_contiguous(const pkv_attn_desc *desc, const void *q, cons
     if (st) return st;
     if (desc->dtype != PKV_F16 && desc->dtype != PKV_BF16)
         return fail(PKV_ERR_UNSUPPORTED, "%s: 16-bit caches only (f16, bf16)", fn);
-    const int64_t lmax = (int64_t)desc->max_blocks_per_seq * pkv::kBlock;
+    const int64_t lmax = (int64_t)desc->max_blocks_per_seq * desc->block_size;
     if ((int64_t)desc->num_seqs * desc->num_kv_heads * lmax >= ((int64_t)1 << 31))
         return fail(PKV_ERR_UNSUPPORTED, "%s: cache too large for 32-bit TMA rows", fn);
     if (desc->num_seqs == 0) return PKV_OK;
@@ -477,6 +486,7 @@ pkv_status attn_decode_contiguous(const pkv_attn_desc *desc, const void *q, cons
     prm.part_blocks = sp.part_blocks;
     prm.pmax = sp.pmax;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.bshift = block_shift(desc);
     prm.Lmax = (int32_t)lmax;
     const int g = desc->num_q_heads / desc->num_kv_heads;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -536,7 +546,8 @@ pkv_status launch_decode_fp8(const pkv::DecodeFp8Params &fp, cudaStream_t stream
     pkv_status st = ensure_smem(kern, kSmem, done, "paged_attn_decode_fp8");
     if (st) return st;
     CUtensorMap tmk;
-    st = fp8_k_tensor_map(&tmk, fp.base.k_pool, (int64_t)fp.base.NB * fp.base.Hkv * pkv::kBlock,
+    st = fp8_k_tensor_map(&tmk, fp.base.k_pool,
+                          ((int64_t)fp.base.NB * fp.base.Hkv) << fp.base.bshift,
                           "paged_attn_decode_fp8");
     if (st) return st;
     const unsigned grid = (unsigned)((int64_t)fp.base.S * fp.base.Hkv * fp.base.pmax);
@@ -578,7 +589,7 @@ Split fp8_split(const pkv_attn_desc *d, const Split &dflt) {
     if (slots <= 0 || pairs < 4 * slots) return dflt;
     Split sp;
     sp.part_blocks = kFp8WidePartitionTokens / pkv::kBlock;
-    sp.pmax = (d->max_blocks_per_seq + sp.part_blocks - 1) / sp.part_blocks;
+    sp.pmax = (sub_blocks_per_seq(d) + sp.part_blocks - 1) / sp.part_blocks;
     return sp.pmax < dflt.pmax ? sp : dflt;
 }
 
@@ -608,7 +619,7 @@ pkv_status decode_fp8_impl(const pkv_attn_desc *desc, const void *q, const void 
         return fail(PKV_ERR_UNSUPPORTED, "%s: q/out must be f16 or bf16", fn);
     if (desc->head_dim != 128)
         return fail(PKV_ERR_UNSUPPORTED, "%s: only head_dim 128 is built", fn);
-    if ((int64_t)desc->num_blocks * desc->num_kv_heads * pkv::kBlock >= ((int64_t)1 << 31))
+    if ((int64_t)desc->num_blocks * desc->num_kv_heads * desc->block_size >= ((int64_t)1 << 31))
         return fail(PKV_ERR_UNSUPPORTED, "%s: pool too large for 32-bit TMA rows", fn);
     if (desc->num_seqs == 0) return PKV_OK;
     if (!q || !k_pool || !v_pool || !k_scale || !v_scale || !block_tables || !context_lens ||
@@ -652,6 +663,7 @@ pkv_status decode_fp8_impl(const pkv_attn_desc *desc, const void *q, const void 
     prm.part_blocks = run.part_blocks;
     prm.pmax = run.pmax;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.bshift = block_shift(desc);
     fp.k_scale = k_scale;
     fp.v_scale = v_scale;
     const int g = desc->num_q_heads / desc->num_kv_heads;
@@ -701,6 +713,7 @@ pkv_status kv_write_fp8(const pkv_attn_desc *desc, const void *k_new, const void
     prm.Hkv = desc->num_kv_heads;
     prm.NB = desc->num_blocks;
     prm.D = desc->head_dim;
+    prm.bshift = block_shift(desc);
     dim3 grid;
     st = write_grid(num_tokens, (int64_t)prm.Hkv * (prm.D / 2), &grid, fn);
     if (st) return st;
@@ -838,7 +851,7 @@ pkv_status launch_swap(const pkv_attn_desc *desc, const int32_t *pairs, int32_t 
     prm.P = n;
     prm.nb_src = nb_src;
     prm.nb_dst = nb_dst;
-    prm.vpb = (int64_t)desc->num_kv_heads * pkv::kBlock * desc->head_dim *
+    prm.vpb = (int64_t)desc->num_kv_heads * desc->block_size * desc->head_dim *
               elem_size(desc->dtype) / 16;
     const int64_t slices = (prm.vpb + pkv::kCopyUnroll * 256 - 1) / (pkv::kCopyUnroll * 256);
     if (slices > 65535) return fail(PKV_ERR_UNSUPPORTED, "%s: block too large", fn);

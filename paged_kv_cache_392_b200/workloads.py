@@ -87,19 +87,20 @@ def _slots(lens, bt, block_size=BLOCK_SIZE):
 
 def make_workload(name, lens, num_q_heads, num_kv_heads, head_dim, dtype, seed,
                   pool_factor=1.1, num_blocks=None, partition_tokens=0, q_std=1.0,
-                  kv_std=0.5, rng=None, max_blocks=None):
+                  kv_std=0.5, rng=None, max_blocks=None, block_size=BLOCK_SIZE):
     rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
     lens = np.asarray(lens, np.int32)
-    need = int(((lens.astype(np.int64) + BLOCK_SIZE - 1) // BLOCK_SIZE).sum())
+    need = int(((lens.astype(np.int64) + block_size - 1) // block_size).sum())
     if num_blocks is None:
         num_blocks = max(1, int(math.ceil(pool_factor * need)))
-    bt, order = _tables(lens, num_blocks, rng, max_blocks=max_blocks)
+    bt, order = _tables(lens, num_blocks, rng, block_size=block_size, max_blocks=max_blocks)
     return Workload(name=name, num_seqs=len(lens), num_q_heads=num_q_heads,
                     num_kv_heads=num_kv_heads, head_dim=head_dim, dtype=dtype,
                     context_lens=lens, block_tables=bt, num_blocks=num_blocks,
-                    free_order=order, slot_mapping=_slots(lens, bt),
+                    free_order=order, slot_mapping=_slots(lens, bt, block_size),
                     scale=1.0 / math.sqrt(head_dim), seed=seed,
-                    partition_tokens=partition_tokens, q_std=q_std, kv_std=kv_std)
+                    partition_tokens=partition_tokens, q_std=q_std, kv_std=kv_std,
+                    block_size=block_size)
 
 
 def tiny():
@@ -107,21 +108,23 @@ def tiny():
                          kv_std=1.0)
 
 
-def opt13b(num_seqs=64, seed=1):
+def opt13b(num_seqs=64, seed=1, block_size=BLOCK_SIZE):
     rng = np.random.Generator(np.random.PCG64(seed))
     lens = np.clip(np.rint(rng.lognormal(math.log(512.0), 1.0, num_seqs)), 16, 2048)
-    return make_workload("opt13b", lens.astype(np.int32), 40, 40, 128, "f16", seed, rng=rng)
+    return make_workload("opt13b", lens.astype(np.int32), 40, 40, 128, "f16", seed, rng=rng,
+                         block_size=block_size)
 
 
-def gqa(num_seqs=128, seed=2):
+def gqa(num_seqs=128, seed=2, block_size=BLOCK_SIZE):
     rng = np.random.Generator(np.random.PCG64(seed))
     lens = rng.integers(256, 4096, size=num_seqs, endpoint=True)
-    return make_workload("gqa", lens.astype(np.int32), 32, 8, 128, "bf16", seed, rng=rng)
+    return make_workload("gqa", lens.astype(np.int32), 32, 8, 128, "bf16", seed, rng=rng,
+                         block_size=block_size)
 
 
-def long_context(num_seqs=8, seq_len=32768, seed=4):
+def long_context(num_seqs=8, seq_len=32768, seed=4, block_size=BLOCK_SIZE):
     return make_workload("long", [seq_len] * num_seqs, 32, 8, 128, "bf16", seed,
-                         partition_tokens=512)
+                         partition_tokens=512, block_size=block_size)
 
 
 # fork / parallel-sampling workload parameters (block tables come from a block manager)
@@ -207,7 +210,8 @@ def fp8_scales(wl, which):
 def make_values_fp8(wl, device="cpu", torch=None):
     """Inputs for an FP8 KV cache: q and new K/V as for ``make_values`` (in wl.dtype); the
     pools as random E4M3 codes of N(0, kv_std^2) values at the per-head scales,
-    K [NB, Hkv, 16, D] and V [NB, Hkv, D, 16]; scales as fp32 tensors."""
+    K [NB, Hkv, B, D] and V [NB, Hkv, D, 16] (16-token blocks) or [NB, Hkv, B/16, D, 16];
+    scales as fp32 tensors."""
     if torch is None:
         import torch  # noqa: F811
     vals = make_values(wl, device, torch)
@@ -224,7 +228,9 @@ def make_values_fp8(wl, device="cpu", torch=None):
         return x.to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
 
     vals["k_pool"] = codes((NB, Hkv, wl.block_size, D), ks, base + 6, 1)
-    vals["v_pool"] = codes((NB, Hkv, D, wl.block_size), vs, base + 7, 1)
+    # V: each 16-token half of a block transposed ([NB, Hkv, D, 16] for 16-token blocks)
+    vshape = (NB, Hkv, D, 16) if wl.block_size == 16 else (NB, Hkv, wl.block_size // 16, D, 16)
+    vals["v_pool"] = codes(vshape, vs, base + 7, 1)
     vals["k_scale"] = ks
     vals["v_scale"] = vs
     return vals

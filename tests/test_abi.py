@@ -66,7 +66,7 @@ def test_workspace_bytes(lib):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(head_dim=96), 3), (dict(block_size=32), 3), (dict(num_q_heads=6), 3),
+    (dict(head_dim=96), 3), (dict(block_size=24), 3), (dict(num_q_heads=6), 3),
     (dict(num_q_heads=7), 1), (dict(dtype=9), 1), (dict(num_blocks=0), 1),
     (dict(partition_tokens=100), 1), (dict(max_blocks_per_seq=0), 1),
     (dict(num_seqs=-1), 1), (dict(dtype=0, head_dim=128, num_q_heads=16), 3),

@@ -24,13 +24,13 @@ def same_state(bm, model, seqs):
         assert bm.seq_len(s) == model.seq_len(s)
 
 
-@pytest.mark.parametrize("seed", [0, 1, 2])
-def test_random_traffic_matches_model(seed):
+@pytest.mark.parametrize("seed,block_size", [(0, 16), (1, 16), (2, 16), (3, 32), (4, 32)])
+def test_random_traffic_matches_model(seed, block_size):
     rng = np.random.default_rng(seed)
-    NB = 48
+    NB = 48 if block_size == 16 else 30
     order = rng.permutation(NB)
-    bm = B.BlockManager(NB, free_order=order)
-    model = BlockManagerModel(NB, free_order=order)
+    bm = B.BlockManager(NB, block_size=block_size, free_order=order)
+    model = BlockManagerModel(NB, block_size=block_size, free_order=order)
     live, nxt = [], 100
     for _ in range(1500):
         op = int(rng.integers(0, 12))
@@ -145,7 +145,7 @@ def test_errors_leave_state_unchanged():
     with pytest.raises(B.PkvError):
         B.BlockManager(4, free_order=[0, 1, 1, 2])
     with pytest.raises(B.PkvError):
-        B.BlockManager(4, block_size=32)
+        B.BlockManager(4, block_size=24)
 
 
 def test_packed_tables():

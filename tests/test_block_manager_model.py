@@ -90,10 +90,11 @@ def test_out_of_blocks_changes_nothing():
                      dict(bm.lens))
 
 
-def test_random_traffic_invariants():
+@pytest.mark.parametrize("B", [16, 32])
+def test_random_traffic_invariants(B):
     rng = np.random.default_rng(7)
     NB = 64
-    bm = BlockManagerModel(NB, 16, free_order=rng.permutation(NB))
+    bm = BlockManagerModel(NB, B, free_order=rng.permutation(NB))
     live, nxt = [], 0
     for step in range(3000):
         op = rng.integers(0, 10)
@@ -124,7 +125,7 @@ def test_random_traffic_invariants():
         assert sorted(bm.free_order()) == [b for b in range(NB) if count[b] == 0]
         # only the last block of a sequence is partly empty
         for s in live:
-            assert 0 <= bm.waste(s) < 16 or bm.seq_len(s) == 0
+            assert 0 <= bm.waste(s) < B or bm.seq_len(s) == 0
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
