@@ -665,7 +665,7 @@ def run_pkv(args):
     pairs_d = torch.from_numpy(np.ascontiguousarray(pairs, np.int32)).to(device)
     out = torch.empty_like(q)
     desc = B.make_desc(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                       wl.num_blocks, bt.shape[1], q.dtype, pt or 0)
+                       wl.num_blocks, bt.shape[1], q.dtype, pt or 0, wl.block_size)
     ws_bytes = B.attn_workspace_bytes(desc)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     npairs = len(pairs)
