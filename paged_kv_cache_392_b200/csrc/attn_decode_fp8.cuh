@@ -117,23 +117,23 @@ __device__ __forceinline__ __nv_fp8x2_storage_t quantize2(const void *src, int64
 // A slot of -1 is skipped; any slot other than position L-1's sets fault bit 4 (bad slot)
 // and is not written, and neither is anything when the head's K or V scale is not finite
 // and > 0 (fault bit 0x40).
-template <typename T>
+template <typename T, int BSH>
 __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp, int s, int hk,
                                                        int L, int lane) {
     constexpr int D = 128;
     const DecodeParams &p = fp.base;
     const int64_t slot = p.slot_mapping[s];
     if (slot != -1) {
-        const int32_t blk = p.block_tables[(size_t)s * p.maxB + ((L - 1) >> p.bshift)];
-        const int off = (L - 1) & ((1 << p.bshift) - 1);
+        const int32_t blk = p.block_tables[(size_t)s * p.maxB + ((L - 1) >> BSH)];
+        const int off = (L - 1) & ((1 << BSH) - 1);
         const float ksc = fp.k_scale[hk], vsc = fp.v_scale[hk];
         if (!scale_ok(ksc) || !scale_ok(vsc)) {
             if (lane == 0) atomicOr(&g_faults, kFaultBadScale);
-        } else if ((unsigned)blk < (unsigned)p.NB && slot == ((int64_t)blk << p.bshift) + off) {
+        } else if ((unsigned)blk < (unsigned)p.NB && slot == ((int64_t)blk << BSH) + off) {
             const int64_t src = ((int64_t)s * p.Hkv + hk) * D;
             const int64_t hb = (int64_t)blk * p.Hkv + hk;
             // the 16-token half of the block that holds the token, and its V^T slot
-            const int64_t vh = (hb << (p.bshift - 4)) + (off >> 4);
+            const int64_t vh = (hb << (BSH - 4)) + (off >> 4);
             const int vs = v_slot_of_token(off & 15);
             // the pools are written only here; the decode itself reads them
             uint8_t *kp = static_cast<uint8_t *>(const_cast<void *>(p.k_pool));
@@ -141,7 +141,7 @@ __device__ __forceinline__ void write_newest_token_fp8(const DecodeFp8Params &fp
             for (int d = 2 * lane; d < D; d += 64) {
                 const __nv_fp8x2_storage_t kc = quantize2<T>(p.k_new, src + d, ksc);
                 const __nv_fp8x2_storage_t vc = quantize2<T>(p.v_new, src + d, vsc);
-                *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + ((hb << p.bshift) + off) * D +
+                *reinterpret_cast<__nv_fp8x2_storage_t *>(kp + ((hb << BSH) + off) * D +
                                                           d) = kc;
                 vp[(vh * D + d) * kBlock + vs] = static_cast<uint8_t>(vc & 0xffu);
                 vp[(vh * D + d + 1) * kBlock + vs] = static_cast<uint8_t>(vc >> 8);
@@ -182,8 +182,10 @@ struct DecodeFp8Cfg {
 constexpr int kFp8WarpsPerSm = PKV_FP8_WARPS_PER_SM;
 
 // T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.  G query heads
-// per kv head, W warps per CTA, NSW ring stages per warp.
-template <typename T, int G, int W, int NSW>
+// per kv head, W warps per CTA, NSW ring stages per warp, BSH log2 of the tokens per physical
+// block (4 or 5: a compile-time constant here, so that the block addressing of the 16-token
+// blocks costs this instruction-bound kernel nothing; it must equal DecodeParams::bshift).
+template <typename T, int G, int W, int NSW, int BSH>
 __global__ void __launch_bounds__(W * 32, kFp8WarpsPerSm / W)
 paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                              const DecodeFp8Params fp) {
@@ -205,7 +207,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     const int s = rest / p.Hkv;
 
     const int L = p.context_lens[s];
-    if (L < 1 || L > (p.maxB << p.bshift)) {
+    if (L < 1 || L > (p.maxB << BSH)) {
         if (part == 0 && hk == 0 && threadIdx.x == 0) atomicOr(&g_faults, kFaultBadLen);
         return;
     }
@@ -234,20 +236,20 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     }
     __syncwarp();
     if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
-        write_newest_token_fp8<T>(fp, s, hk, L, lane);
+        write_newest_token_fp8<T, BSH>(fp, s, hk, L, lane);
 
     const int32_t *btab = p.block_tables + (size_t)s * p.maxB;
     const int j1 = j0 + warp;  // this warp's first sub-block
     const char *vbase = static_cast<const char *>(p.v_pool);
     const uint64_t policy = l2_evict_first_policy();
     int tab_chunk = 0;
-    int32_t tab = lane < nbw ? btab[sub_to_entry(j1 + W * lane, p.bshift)] : 0;
+    int32_t tab = lane < nbw ? btab[sub_to_entry(j1 + W * lane, BSH)] : 0;
 
     auto issue = [&](int i) {
         if ((i >> 5) != tab_chunk) {
             tab_chunk = i >> 5;
             const int li = (tab_chunk << 5) + lane;
-            tab = li < nbw ? btab[sub_to_entry(j1 + W * li, p.bshift)] : 0;
+            tab = li < nbw ? btab[sub_to_entry(j1 + W * li, BSH)] : 0;
         }
         const int32_t phys = __shfl_sync(FULL, tab, i & 31);
         if (lane == 0 && !withheld_for_test(i, warp)) {
@@ -255,11 +257,11 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
             unsigned char *dst = ring + (i % NSW) * C::STAGE;
             if ((unsigned)phys < (unsigned)p.NB) {
                 const int jb = j1 + W * i;
-                const int32_t row = ((phys * p.Hkv + hk) << p.bshift) + sub_row(jb, p.bshift);
+                const int32_t row = ((phys * p.Hkv + hk) << BSH) + sub_row(jb, BSH);
                 // V^T of the sub-block: the 16-token half (jb's position in the block) of
                 // the block's [B/16][D][16] bytes
-                const size_t vhalf = ((size_t)(phys * p.Hkv + hk) << (p.bshift - 4)) +
-                                     (size_t)(sub_row(jb, p.bshift) / kBlock);
+                const size_t vhalf = ((size_t)(phys * p.Hkv + hk) << (BSH - 4)) +
+                                     (size_t)(sub_row(jb, BSH) / kBlock);
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(bar, 2 * CHUNK);
                 tma_load_2d(dst, &tmk, 0, row, bar, policy);

@@ -536,12 +536,12 @@ pkv_status fp8_k_tensor_map(CUtensorMap *m, const void *pool, int64_t rows, cons
     return PKV_OK;
 }
 
-template <typename T, int G>
+template <typename T, int G, int BSH>
 pkv_status launch_decode_fp8(const pkv::DecodeFp8Params &fp, cudaStream_t stream) {
     constexpr int kW = fp8_warps<G>();
     using Cfg = pkv::DecodeFp8Cfg<kW, kFp8Stages>;
     constexpr int kSmem = Cfg::template smem<G>();
-    auto kern = pkv::paged_attn_decode_fp8_kernel<T, G, kW, kFp8Stages>;
+    auto kern = pkv::paged_attn_decode_fp8_kernel<T, G, kW, kFp8Stages, BSH>;
     static std::atomic<bool> done[kMaxDevices];
     pkv_status st = ensure_smem(kern, kSmem, done, "paged_attn_decode_fp8");
     if (st) return st;
@@ -555,6 +555,13 @@ pkv_status launch_decode_fp8(const pkv::DecodeFp8Params &fp, cudaStream_t stream
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode_fp8", "decode launch");
     return launch_reduce_if_split(fp.base, stream, pkv::lse_reduce_kernel<T, 128>);
+}
+
+// The FP8 kernel takes the block size as a template parameter (16- or 32-token blocks).
+template <typename T, int G>
+pkv_status launch_decode_fp8_bs(const pkv::DecodeFp8Params &fp, cudaStream_t stream) {
+    return fp.base.bshift == 5 ? launch_decode_fp8<T, G, 5>(fp, stream)
+                               : launch_decode_fp8<T, G, 4>(fp, stream);
 }
 
 // Streaming multiprocessors of the current device (looked up once per device).
@@ -596,10 +603,10 @@ Split fp8_split(const pkv_attn_desc *d, const Split &dflt) {
 template <typename T>
 pkv_status dispatch_fp8(int g, const pkv::DecodeFp8Params &fp, cudaStream_t stream) {
     switch (g) {
-    case 1: return launch_decode_fp8<T, 1>(fp, stream);
-    case 2: return launch_decode_fp8<T, 2>(fp, stream);
-    case 4: return launch_decode_fp8<T, 4>(fp, stream);
-    case 8: return launch_decode_fp8<T, 8>(fp, stream);
+    case 1: return launch_decode_fp8_bs<T, 1>(fp, stream);
+    case 2: return launch_decode_fp8_bs<T, 2>(fp, stream);
+    case 4: return launch_decode_fp8_bs<T, 4>(fp, stream);
+    case 8: return launch_decode_fp8_bs<T, 8>(fp, stream);
     default: return fail(PKV_ERR_UNSUPPORTED, "paged_attn_decode_fp8: group %d", g);
     }
 }
