@@ -787,6 +787,7 @@ def run_pkv(args):
         barrier(dist, device)
         torch.cuda.synchronize()
         sampler.start()
+        torch.cuda.nvtx.range_push("timed steps")
         t0.record(gs)
         if g_rem is not None:
             g_rem.replay()
@@ -797,6 +798,7 @@ def run_pkv(args):
             rep_ev[r].record(gs)
         t1.record(gs)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
         barrier(dist, device)
     sampler.stop()
     ms_local = t0.elapsed_time(t1)
@@ -911,25 +913,31 @@ def run_pkv(args):
     barrier(dist, device)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("e2e serial")
     e0.record(main)
     for _ in range(Ks):
         e2e_serial_step()
     e1.record(main)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     e2e_serial_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ks, device)
     barrier(dist, device)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("e2e pipelined")
     e0.record(main)
     e2e_pipelined(Ke)
     e1.record(main)                # e2e_pipelined returned after the last output landed
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ke, device)
     barrier(dist, device)
     faults = B.device_faults(clear=True)
     if faults:
         raise RuntimeError("device faults during the end-to-end runs: %s" % faults)
+    torch.cuda.nvtx.range_push("kv_write / kv_copy_blocks alone")
     aux = time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ksc, vsc,
                            nbytes)
+    torch.cuda.nvtx.range_pop()
     faults = B.device_faults(clear=True)
     if faults:
         raise RuntimeError("device faults in the kv_write / kv_copy_blocks timing: %s" % faults)
