@@ -903,9 +903,10 @@ def run_pkv(args):
         d2h_stream.synchronize()
         main.synchronize()
 
-    # pipelined e2e: at least 200 steps, so that the two-deep pipeline's fill and drain and the
-    # first replays of the freshly captured graphs do not dominate a short run
-    Ke = max(200, K)
+    # pipelined e2e: at least 1000 steps (about 0.13 s on the headline batch), so that the
+    # two-deep pipeline's fill and drain and the first replays of the freshly captured graphs
+    # do not dominate a short run
+    Ke = max(1000, K)
     Ks = max(1, min(K, 1000))     # serial mode: at most 1000 synchronised steps
     for _ in range(max(3, args.warmup // 4)):
         e2e_serial_step()
