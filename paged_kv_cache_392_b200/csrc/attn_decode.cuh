@@ -25,6 +25,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "faults.cuh"
 #include "ptx.cuh"
@@ -560,24 +561,69 @@ paged_attn_decode_kernel(const DecodeParams p) {
 
 // ---- log-sum-exp merge of the partitions of split sequences ----------------------------
 // out[s,h,:] = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p  (base-2 units,
-// which is the natural-log formula with every logit scaled by log2(e)).  One CTA of four
-// warps per (sequence, query head) row: the warps take every fourth partition, each lane a
-// D/32-float slice of o_p (vector loads, unrolled so several partitions are in flight), and
-// the four partial sums meet in shared memory.  Rows whose sequence fits in one partition
-// were already written by the decode kernel.
-constexpr int kReduceWarps = 4;
+// which is the natural-log formula with every logit scaled by log2(e)).  The kernel reads a
+// few KB a row from L2 right after the decode wrote them, so its time is round trips, and it
+// is built to take as few as possible:
+//   * R warps per (sequence, query head) row: one when no row has more than kReduceBatch
+//     partitions (four rows to a CTA), else kReduceWideWarps (one row to a CTA);
+//   * warp w of a row takes partitions w, w+R, w+2R, ... in batches of kReduceBatch whose
+//     (m, l) pairs and o_p slices (a D/32-float slice per lane) are all loaded before the
+//     first is used, so a row of up to R * kReduceBatch partitions costs one round trip;
+//   * each warp keeps its own running max (rescaling its sums when a batch raises it), and
+//     with R > 1 the warps' states meet in shared memory under the same merge formula.
+// A partition whose m is -inf (no state) weighs 0; a row with no state at all comes out NaN.
+// Rows whose sequence fits in one partition were already written by the decode kernel.
+constexpr int kReduceBatch = 8;
+constexpr int kReduceWideWarps = 8;
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const DecodeParams p) {
-    constexpr int NW = kReduceWarps;
+template <int VL>
+struct ReduceVec;
+template <>
+struct ReduceVec<2> {
+    using type = float2;
+    __device__ static float get(const float2 &v, int k) { return k == 0 ? v.x : v.y; }
+};
+template <>
+struct ReduceVec<4> {
+    using type = float4;
+    __device__ static float get(const float4 &v, int k) {
+        return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+    }
+};
+
+// N floats to N consecutive elements of T (one 4-, 8- or 16-byte store).
+template <typename T, int N>
+__device__ __forceinline__ void store_vec(T *dst, const float (&x)[N]) {
+    constexpr int kBytes = N * (int)sizeof(T);
+    static_assert(kBytes == 4 || kBytes == 8 || kBytes == 16, "one 4/8/16-byte vector");
+    using V = typename std::conditional<
+        kBytes == 16, uint4, typename std::conditional<kBytes == 8, uint2, uint32_t>::type>::type;
+    union {
+        V v;
+        T e[N];
+    } u;
+#pragma unroll
+    for (int i = 0; i < N; ++i) u.e[i] = Elem<T>::from_float(x[i]);
+    *reinterpret_cast<V *>(dst) = u.v;
+}
+
+template <typename T, int D, int R>
+__global__ void __launch_bounds__(R == 1 ? 128 : R * 32) lse_reduce_kernel(const DecodeParams p) {
+    constexpr int U = kReduceBatch;
     constexpr int VL = D / 32;             // floats per lane
-    constexpr int E = 16 / sizeof(T);      // output elements per 16-byte store
-    __shared__ float s_m[NW];
-    __shared__ float s_den[NW];
-    __shared__ __align__(16) float s_acc[NW][D];
+    using V = ReduceVec<VL>;
+    using VT = typename V::type;
+    constexpr int NS = R == 1 ? 1 : R;     // shared-memory states (unused with R == 1)
+    __shared__ float s_m[NS];
+    __shared__ float s_den[NS];
+    __shared__ __align__(16) float s_acc[NS][D];
 
     pdl_wait_primary();
-    const int row = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // R == 1: warp-uniform row; R > 1: CTA-uniform row (so the returns below keep every
+    // warp of a CTA that reaches the barrier together)
+    const int row = R == 1 ? blockIdx.x * 4 + warp : blockIdx.x;
+    const int wr = R == 1 ? 0 : warp;      // the warp's index within its row
     if (row >= p.S * p.Hq) return;
     const int s = row / p.Hq;
     const int L = p.context_lens[s];
@@ -585,58 +631,82 @@ __global__ void __launch_bounds__(kReduceWarps * 32) lse_reduce_kernel(const Dec
     const int nblk = (L + kBlock - 1) / kBlock;
     const int np = (nblk + p.part_blocks - 1) / p.part_blocks;
     if (np <= 1) return;
-    const float *ml = p.ws_ml + (size_t)row * p.pmax * 2;
-    const float *ob = p.ws_o + (size_t)row * p.pmax * D;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.ws_ml) + (size_t)row * p.pmax;
+    const float *ob = p.ws_o + (size_t)row * p.pmax * D + lane * VL;
 
-    float M = -INFINITY;
-    for (int i = threadIdx.x; i < np; i += NW * 32) M = fmaxf(M, ml[2 * i]);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-    if (lane == 0) s_m[warp] = M;
-    __syncthreads();
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_m[w]);
-
-    float acc[VL], den = 0.f;
+    float M = -INFINITY, den = 0.f, acc[VL];
 #pragma unroll
     for (int k = 0; k < VL; ++k) acc[k] = 0.f;
-#pragma unroll 4
-    for (int i = warp; i < np; i += NW) {
-        const float w = exp2f(ml[2 * i] - M);
-        den = fmaf(w, ml[2 * i + 1], den);
-        const float *src = ob + (size_t)i * D + lane * VL;
-        if constexpr (VL == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(src);
-            acc[0] = fmaf(w, v.x, acc[0]);
-            acc[1] = fmaf(w, v.y, acc[1]);
-            acc[2] = fmaf(w, v.z, acc[2]);
-            acc[3] = fmaf(w, v.w, acc[3]);
-        } else {
-            const float2 v = *reinterpret_cast<const float2 *>(src);
-            acc[0] = fmaf(w, v.x, acc[0]);
-            acc[1] = fmaf(w, v.y, acc[1]);
+    for (int i0 = wr; i0 < np; i0 += R * U) {
+        float2 mlv[U];
+        VT v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + R * u;
+            if (i < np) {
+                mlv[u] = ml[i];
+                v[u] = *reinterpret_cast<const VT *>(ob + (size_t)i * D);
+            } else {
+                mlv[u] = make_float2(-INFINITY, 0.f);
+            }
+        }
+        float bm = M;
+#pragma unroll
+        for (int u = 0; u < U; ++u) bm = fmaxf(bm, mlv[u].x);
+        if (bm > M) {  // the batch raises the running max: rescale what is summed so far
+            const float a = M == -INFINITY ? 0.f : exp2f(M - bm);
+            den *= a;
+#pragma unroll
+            for (int k = 0; k < VL; ++k) acc[k] *= a;
+            M = bm;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (mlv[u].x != -INFINITY) {
+                const float w = exp2f(mlv[u].x - M);
+                den = fmaf(w, mlv[u].y, den);
+#pragma unroll
+                for (int k = 0; k < VL; ++k) acc[k] = fmaf(w, V::get(v[u], k), acc[k]);
+            }
         }
     }
-#pragma unroll
-    for (int k = 0; k < VL; ++k) s_acc[warp][lane * VL + k] = acc[k];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
 
-    for (int idx = threadIdx.x; idx < D / E; idx += NW * 32) {
-        float dsum = 0.f;
+    if constexpr (R == 1) {
+        const float inv = 1.f / den;
+        float x[VL];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) dsum += s_den[w];
-        const float inv = 1.f / dsum;
-        float v[E];
+        for (int k = 0; k < VL; ++k) x[k] = acc[k] * inv;
+        store_vec<T, VL>(static_cast<T *>(p.out) + (size_t)row * D + lane * VL, x);
+    } else {
+        constexpr int E = 16 / sizeof(T);  // output elements per 16-byte store
 #pragma unroll
-        for (int e = 0; e < E; ++e) {
-            float t = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) t += s_acc[w][idx * E + e];
-            v[e] = t * inv;
+        for (int k = 0; k < VL; ++k) s_acc[warp][lane * VL + k] = acc[k];
+        if (lane == 0) {
+            s_m[warp] = M;
+            s_den[warp] = den;
         }
-        store_row<T, E>(static_cast<T *>(p.out) + (size_t)row * D + idx * E, v);
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < D / E; idx += R * 32) {
+            float Mx = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < R; ++w) Mx = fmaxf(Mx, s_m[w]);
+            float a[R], dsum = 0.f;
+#pragma unroll
+            for (int w = 0; w < R; ++w) {
+                a[w] = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - Mx);
+                dsum = fmaf(a[w], s_den[w], dsum);
+            }
+            const float inv = 1.f / dsum;
+            float x[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                float t = 0.f;
+#pragma unroll
+                for (int w = 0; w < R; ++w) t = fmaf(a[w], s_acc[w][idx * E + e], t);
+                x[e] = t * inv;
+            }
+            store_row<T, E>(static_cast<T *>(p.out) + (size_t)row * D + idx * E, x);
+        }
     }
 }
 

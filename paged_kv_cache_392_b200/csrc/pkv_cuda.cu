@@ -152,12 +152,16 @@ pkv_status kv_tensor_map(CUtensorMap *m, const void *pool, int32_t dtype, int D,
     return PKV_OK;
 }
 
-pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t stream,
-                                  void (*kern)(const pkv::DecodeParams)) {
+// The log-sum-exp reduce after a split decode: one warp per row when no row can have more
+// than kReduceBatch partitions (pmax bounds them all), else kReduceWideWarps warps per row.
+template <typename T, int D>
+pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t stream) {
     if (prm.pmax <= 1) return PKV_OK;
+    const int64_t rows = (int64_t)prm.S * prm.Hq;
+    const bool narrow = prm.pmax <= pkv::kReduceBatch;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((int64_t)prm.S * prm.Hq));
-    cfg.blockDim = dim3(pkv::kReduceWarps * 32);
+    cfg.gridDim = dim3((unsigned)(narrow ? (rows + 3) / 4 : rows));
+    cfg.blockDim = dim3(narrow ? 128 : pkv::kReduceWideWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -165,7 +169,9 @@ pkv_status launch_reduce_if_split(const pkv::DecodeParams &prm, cudaStream_t str
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, prm);
+    cudaError_t e =
+        narrow ? cudaLaunchKernelEx(&cfg, pkv::lse_reduce_kernel<T, D, 1>, prm)
+               : cudaLaunchKernelEx(&cfg, pkv::lse_reduce_kernel<T, D, pkv::kReduceWideWarps>, prm);
     return cuda_check(e, "paged_attn_decode", "reduce launch");
 }
 
@@ -192,7 +198,7 @@ pkv_status launch_decode_tc(const pkv::DecodeParams &prm, int32_t dtype, cudaStr
     kern<<<grid, kTcWarps * 32, Cfg::SMEM, stream>>>(tmk, tmv, prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "decode launch");
-    return launch_reduce_if_split(prm, stream, pkv::lse_reduce_kernel<T, D>);
+    return launch_reduce_if_split<T, D>(prm, stream);
 }
 
 template <typename T, int D, int G>
@@ -206,7 +212,7 @@ pkv_status launch_decode(const pkv::DecodeParams &prm, cudaStream_t stream) {
     kern<<<grid, kWarps * 32, Cfg::SMEM, stream>>>(prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode", "decode launch");
-    return launch_reduce_if_split(prm, stream, pkv::lse_reduce_kernel<T, D>);
+    return launch_reduce_if_split<T, D>(prm, stream);
 }
 
 // Whether the tensor-core kernel serves this call: 16-bit K/V whose 2-D TMA view fits int32
@@ -554,7 +560,7 @@ pkv_status launch_decode_fp8(const pkv::DecodeFp8Params &fp, cudaStream_t stream
     kern<<<grid, kW * 32, kSmem, stream>>>(tmk, fp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_check(e, "paged_attn_decode_fp8", "decode launch");
-    return launch_reduce_if_split(fp.base, stream, pkv::lse_reduce_kernel<T, 128>);
+    return launch_reduce_if_split<T, 128>(fp.base, stream);
 }
 
 // The FP8 kernel takes the block size as a template parameter (16- or 32-token blocks).
