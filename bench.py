@@ -971,8 +971,8 @@ def run_pkv(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("f32 accumulate over fp8-e4m3 KV (q.K on e4m3 tensor-core tiles, "
-                      "P.V on f16 tiles), %s q/out" % wl.dtype) if fp8 else
+            "dtype": ("f32 accumulate over fp8-e4m3 KV (codes widened exactly to f16 for "
+                      "f16 tensor-core tiles), %s q/out" % wl.dtype) if fp8 else
                      "f32 accumulate over %s KV" % wl.dtype,
             "data": "synthetic (seeded), no weights",
             "seqs_per_s": round(world * wl.num_seqs / (step_ms * 1e-3), 1),

@@ -242,10 +242,10 @@ pkv_status kv_swap_in(const pkv_attn_desc *desc, const int32_t *pairs, int32_t n
  * (PKV_F16 or PKV_BF16); the same workspace rule (pkv_attn_workspace_bytes(desc)).  With
  * desc->partition_tokens 0 it may split contexts more coarsely than the 16-bit decode;
  * pkv_fp8_partition_tokens(desc) reports the partition it uses.
- * Scores run on E4M3 tensor-core tiles straight from the K codes (q split into two E4M3
- * terms, about bfloat16 precision); the weighted sum runs on f16 tiles with the V codes
- * widened exactly; accumulation is fp32.  The K scale multiplies the scores and the V scale
- * the output.  Results stay within the q dtype's tolerance of the exact attention over the
+ * Both products run on f16 tensor-core tiles with the K and V codes widened exactly to f16
+ * (every E4M3 value is an f16 value) and q rounded to f16 (exact for an f16 q; a bf16 q is
+ * first scaled by a power of two, so only values 2^-28 below its row's largest lose bits);
+ * accumulation is fp32.  The K scale multiplies the scores and the V scale the output.  Results stay within the q dtype's tolerance of the exact attention over the
  * dequantised codes (2e-3 for f16, 1e-2 for bf16).
  */
 /*

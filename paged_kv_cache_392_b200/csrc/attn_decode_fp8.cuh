@@ -11,13 +11,11 @@
 //     transposed, and slot p of a row holds token 2*(p>>2) + (p&1) + 8*((p>>1)&1) of the
 //     half (v_slot_of_token below is the inverse), so that the 4 bytes an ldmatrix lane
 //     reads from a row are the token pairs the P.V tile wants.
-// Decode: q.K^T runs on m16n8k32 E4M3 tensor-core tiles straight from the K codes, with each
-// query row prescaled by a power of two and split into two E4M3 terms (hi + residual, about
-// bfloat16 precision; with at most four query heads per kv head both terms ride in one MMA
-// chain, side by side in the n columns); P.V widens the V codes exactly to f16 (every E4M3
-// value is an f16 value, scaled by 2^-8 on the integer path) for m16n8k16 f16 tiles.
-// Accumulation is fp32; the K scale (and the q prescale) is folded into the softmax scale
-// and the V scale into the output.  Only D = 128 is built.
+// Decode: q.K^T and P.V run on m16n8k16 f16 tensor-core tiles.  Every E4M3 value is an f16
+// value, so the K and V codes are widened exactly, four codes (two f16x2 registers) per
+// conversion pair; q enters as f16 (an f16 q as is, a bf16 q scaled by a power of two, which
+// rounds it to f16 exactly).  Accumulation is fp32; the K scale (and the q scale) is folded
+// into the softmax scale and the V scale into the output.  Only D = 128 is built.
 #pragma once
 #include <cuda.h>
 #include <cuda_fp8.h>
@@ -34,48 +32,22 @@ __host__ __device__ __forceinline__ int v_slot_of_token(int t) {
     return 4 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
 }
 
-// Two E4M3 codes of w to an f16x2 register holding each value times 2^-8, with integer
-// operations only: an E4M3 code s.eeee.mmm placed as the f16 s.0eeee.mmm0000000 is the same
-// number scaled by 2^(7-15) = 2^-8, subnormals included (f16 keeps E4M3's subnormal grid
-// scaled by the same power of two).  A byte permute in sign-replicating mode builds
-// [sign(b_hi) x8 : b_hi : sign(b_lo) x8 : b_lo] (prmt selector nibbles with bit 3 set copy the
-// selected byte's sign bit into all 8 bits); shifted left by 7, each half holds eeee.mmm at
-// bits 13..7 and the sign at bit 15, and the mask keeps exactly those bits.  sel picks the
-// pair: 0x9180 for bytes 0 and 1, 0xB3A2 for bytes 2 and 3.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
-    uint32_t t;
-    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(t) : "r"(w), "r"(sel));
-    return (t << 7) & 0xBF80BF80u;
-}
-
 // Tuning switch of the FP8 decode (the results are the same bits either way): 1 computes
 // the softmax weights before the rescale vote resolves (measured +0.4 to +1.4 %).
 #ifndef PKV_FP8_SPEC_EXP
 #define PKV_FP8_SPEC_EXP 1
 #endif
 
-// How many of the 8 P.V m-tiles (16 head dims each) widen V on the conversion unit (XU
-// pipe, exact values); the others use the integer trick above (ALU pipe, values x 2^-8).
-// With the three-operation integer form, none on the conversion unit measured fastest.
-#ifndef PKV_FP8_CVT_TILES
-#define PKV_FP8_CVT_TILES 0
-#endif
-constexpr int kCvtTiles = PKV_FP8_CVT_TILES;
-
-// Two E4M3 codes (low byte first) to an f16x2 register, exactly, on the conversion unit.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-}
-
-// D = A * B + C for one m16n8k32 tile of E4M3 codes, fp32 accumulators.
-__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Four E4M3 codes (bytes 0..3 of w) to two f16x2 registers, exactly: lo = codes 0, 1 and
+// hi = codes 2, 3, each pair with its lower-addressed code in the low half.  The conversion
+// reads the 16-bit halves of w directly (one instruction per output register).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // Two floats to an f16x2 register (round to nearest even).
@@ -277,25 +249,21 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     for (int i = 0; i < npro; ++i) issue(i);
     int issued = npro;
 
-    // Q^T as the B operand of S^T = K Q^T on E4M3 tiles (m16n8k32): each query row is scaled
-    // by a power of two qf (its largest |q| lands in [128, 256)) and split into two E4M3
-    // terms, hi = e4m3(q*qf) and lo = e4m3(q*qf - hi), which carry about 8 significant bits
-    // (a bfloat16 q exactly, up to subnormal tails).  Lane (g, tq) holds head g, dims
-    // 32j+4tq..+3 (b0) and 32j+16+4tq..+3 (b1) of k-step j.
-    // With at most four query heads per kv head the two terms share one MMA chain: column n
-    // of the B operand holds the high term of head n (n < G) or the residual of head n - G
-    // (G <= n < 2G), and the two columns of a head are added after the chain.  Each column's
-    // sum is the one the separate chains computed, so the scores are the same bits; the
-    // E4M3 tiles cost about a dozen instructions each on this path, and this halves them.
+    // Q^T as the B operand of S^T = K Q^T on f16 tiles (m16n8k16).  A K register from the
+    // swizzled stage holds 4 consecutive dims of one token (the A fragment of an E4M3
+    // m16n8k32 tile: lane (g, tq) reads dims 32j+4tq.. and 32j+16+4tq.. of tokens g and
+    // g+8); widened, its dims d, d+1 and d+2, d+3 fill the f16 tile's k slots (2tq, 2tq+1)
+    // and (2tq+8, 2tq+9).  The B fragment holds q at the same dims, so each tile sums q.k
+    // over the 16 dims it covers: lane (g, tq) holds head g, dims 32j+16b+4tq..+3 as
+    // qh[j][b][0] (the first two) and qh[j][b][1].  A bf16 q row is scaled by a power of two
+    // qf (its largest |q| lands in [2^14, 2^15)), so that f16 holds every value exactly
+    // except those 2^-28 below the row's largest; an f16 q is used as is.
     constexpr int K32 = D / 32;
-    constexpr bool kPack = G <= 4;
-    uint32_t qhi[K32][2], qlo[K32][2];
+    uint32_t qh[K32][2][2];
     float qf_mine = 1.f;
     {
-        const bool hv = kPack ? g < 2 * G : g < G;
-        const int qh = kPack && g >= G ? g - G : g;  // head of this lane's B column
-        const T *qrow =
-            static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? qh : 0)) * D;
+        const bool hv = g < G;
+        const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
         float qv[K32][2][4];
         float amax = 0.f;
 #pragma unroll
@@ -314,34 +282,21 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
                     qv[j][b][e] = v;
                     amax = fmaxf(amax, fabsf(v));
                 }
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-        if (amax > 0.f && amax < INFINITY) {
-            int ex;
-            frexpf(amax, &ex);                  // amax < 2^ex
-            qf_mine = ldexpf(1.f, 8 - ex);      // amax * qf in [128, 256)
+        if constexpr (!std::is_same<T, __half>::value) {
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+            if (amax > 0.f && amax < INFINITY) {
+                int ex;
+                frexpf(amax, &ex);                  // amax < 2^ex
+                qf_mine = ldexpf(1.f, 15 - ex);     // amax * qf in [2^14, 2^15)
+            }
         }
 #pragma unroll
         for (int j = 0; j < K32; ++j)
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
-                uint32_t hi = 0u, lo = 0u;
-#pragma unroll
-                for (int e = 0; e < 4; e += 2) {
-                    const float2 x =
-                        make_float2(qv[j][b][e] * qf_mine, qv[j][b][e + 1] * qf_mine);
-                    const __nv_fp8x2_storage_t h2 =
-                        __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
-                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h2, __NV_E4M3);
-                    const float2 r = make_float2(x.x - __half2float(__ushort_as_half(hr.x)),
-                                                 x.y - __half2float(__ushort_as_half(hr.y)));
-                    const __nv_fp8x2_storage_t l2 =
-                        __nv_cvt_float2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
-                    hi |= static_cast<uint32_t>(h2) << (8 * e);
-                    lo |= static_cast<uint32_t>(l2) << (8 * e);
-                }
-                qhi[j][b] = kPack && g >= G ? lo : hi;
-                qlo[j][b] = lo;
+                qh[j][b][0] = f32x2_to_f16x2(qv[j][b][0] * qf_mine, qv[j][b][1] * qf_mine);
+                qh[j][b][1] = f32x2_to_f16x2(qv[j][b][2] * qf_mine, qv[j][b][3] * qf_mine);
             }
     }
 
@@ -414,29 +369,18 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
 #pragma unroll
         for (int t2 = 0; t2 < KSTEPS / 2; ++t2) ldmatrix_x4(vr[t2], vb + (32 * t2 + v_row) * 16);
 
-        // ---- S^T = K Q^T on E4M3 tiles: the high and residual q terms in one chain of K32
-        // (packed columns, G <= 4), or in two
+        // ---- S^T = K Q^T on f16 tiles: per 32-dim step, the tile of dims 32j+4tq.. and the
+        // tile of dims 32j+16+4tq..
         float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (kPack) {
 #pragma unroll
-            for (int j = 0; j < K32; ++j) mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
-            if constexpr (G == 1) {  // columns 0 (high) and 1 (residual) sit in one lane
-                sacc[0] += sacc[1];
-                sacc[2] += sacc[3];
-            } else {                 // the residual columns sit G/2 lanes (G columns) away
+        for (int j = 0; j < K32; ++j)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[e] += __shfl_xor_sync(FULL, sacc[e], G / 2);
+            for (int b = 0; b < 2; ++b) {
+                uint32_t a[4];
+                e4m3x4_to_f16x2x2(ka[j][2 * b], a[0], a[2]);      // token g
+                e4m3x4_to_f16x2x2(ka[j][2 * b + 1], a[1], a[3]);  // token g + 8
+                mma_16816<false>(sacc, a, qh[j][b][0], qh[j][b][1]);
             }
-        } else {
-            float sres[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int j = 0; j < K32; ++j) {
-                mma_16832_e4m3(sacc, ka[j], qhi[j][0], qhi[j][1]);
-                mma_16832_e4m3(sres, ka[j], qlo[j][0], qlo[j][1]);
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[e] += sres[e];
-        }
 
         // ---- online softmax (lane: tokens g, g+8 of heads 2tq, 2tq+1) --------------------
         float x0 = sacc[0] * sl0, x1 = sacc[1] * sl1, x2 = sacc[2] * sl0, x3 = sacc[3] * sl1;
@@ -507,17 +451,8 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t a[4];
-                if (2 * t2 + h < kCvtTiles) {
-                    a[0] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] & 0xffffu));
-                    a[2] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h] >> 16));
-                    a[1] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] & 0xffffu));
-                    a[3] = e4m3x2_to_f16x2(static_cast<uint16_t>(r[2 * h + 1] >> 16));
-                } else {
-                    a[0] = e4m3x2_to_f16x2_scaled(r[2 * h], 0x9180u);
-                    a[2] = e4m3x2_to_f16x2_scaled(r[2 * h], 0xB3A2u);
-                    a[1] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0x9180u);
-                    a[3] = e4m3x2_to_f16x2_scaled(r[2 * h + 1], 0xB3A2u);
-                }
+                e4m3x4_to_f16x2x2(r[2 * h], a[0], a[2]);
+                e4m3x4_to_f16x2x2(r[2 * h + 1], a[1], a[3]);
                 mma_16816<false>(o[2 * t2 + h], a, b0, b1);
             }
         }
@@ -545,14 +480,12 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     }
 
     __syncthreads();  // every warp is done with its ring: the merge states go over it
-    // m-tiles widened on the integer pipe carry V x 2^-8
-    const float vsc_cvt = fp.v_scale[hk], vsc_int = vsc_cvt * 256.f;
+    const float vsc = fp.v_scale[hk];
     const int h0 = 2 * tq, h1 = 2 * tq + 1;
     if (h0 < G) {
         float *dst = mo + (warp * G + h0) * D;
 #pragma unroll
         for (int t = 0; t < KSTEPS; ++t) {
-            const float vsc = t < kCvtTiles ? vsc_cvt : vsc_int;
             dst[16 * t + g] = o[t][0] * vsc;
             dst[16 * t + g + 8] = o[t][2] * vsc;
         }
@@ -565,7 +498,6 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
         float *dst = mo + (warp * G + h1) * D;
 #pragma unroll
         for (int t = 0; t < KSTEPS; ++t) {
-            const float vsc = t < kCvtTiles ? vsc_cvt : vsc_int;
             dst[16 * t + g] = o[t][1] * vsc;
             dst[16 * t + g + 8] = o[t][3] * vsc;
         }

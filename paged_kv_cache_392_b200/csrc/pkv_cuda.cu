@@ -582,7 +582,7 @@ int device_sm_count() {
 }
 
 // The FP8 decode's partition when the caller leaves the choice to the library
-// (partition_tokens 0).  Its per-unit work (the q split into E4M3 terms, the warps' merge)
+// (partition_tokens 0).  Its per-unit work (the q conversion to f16, the warps' merge)
 // weighs more against a unit's blocks than in the 16-bit kernel, so when the batch's
 // (sequence, kv head) pairs alone give at least four CTAs per resident CTA slot it takes
 // units of up to kFp8WidePartitionTokens (one per pair for contexts up to that), else the
