@@ -155,3 +155,25 @@ def test_decode_fp8_full_size_opt13b_every_row():
     print("opt13b fp8 (f16 q): max abs error over all %d rows: %.3e (tolerance %g)"
           % (wl.num_seqs * 40, err, TOL["f16"]))
     assert err <= TOL["f16"], err
+
+
+@pytest.mark.parametrize("gain", [8.0, 32.0])
+def test_decode_fp8_f16_q_enters_exactly(gain):
+    """An f16 q reaches the score tiles unrounded (every E4M3 code and every f16 q value are
+    f16 values, and the products accumulate in fp32).  A sharp softmax, q scaled by 8 or 32,
+    makes the output sensitive to any rounding of q: a q carried with about 8 significant
+    bits moves the scores by ~2^-9 * gain and misses the f16 tolerance, while only the f16
+    weights and the f16 output round here."""
+    wl = W.make_workload("x", [16, 100, 257, 700, 1500], 8, 2, 128, "f16", 77, pool_factor=1.3)
+    v = {k: t.cuda() for k, t in W.make_values_fp8(wl, "cpu").items()}
+    v["q"] = v["q"] * gain                        # a power of two: exact in f16
+    out = B.paged_attn_decode_fp8(v["q"], v["k_pool"], v["v_pool"], v["k_scale"], v["v_scale"],
+                                  torch.from_numpy(wl.block_tables).cuda(),
+                                  torch.from_numpy(wl.context_lens).cuda(), wl.scale)
+    torch.cuda.synchronize()
+    ref = oracle.paged_attn_decode_fp8(bits(v["q"]), u8(v["k_pool"]), u8(v["v_pool"]),
+                                       u8(v["k_scale"]), u8(v["v_scale"]), wl.block_tables,
+                                       wl.context_lens, wl.scale, "f16")
+    err = float(np.max(np.abs(out.double().cpu().numpy() - ref)))
+    print("fp8, f16 q x %g: max abs error %.3e (tolerance %g)" % (gain, err, TOL["f16"]))
+    assert err <= TOL["f16"], err
