@@ -19,6 +19,7 @@ same workload on the host cores.
 """
 import argparse
 import datetime
+import gc
 import hashlib
 import json
 import math
@@ -35,6 +36,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention KV GB/s & seqs/s, % of B200 HBM roofline"
+# Buffer sets of the pipelined end-to-end run (the host runs up to E2E_BUFS - 1 steps ahead)
+E2E_BUFS = 3
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1000 * 1000     # B200 L2 (126 MB)
 
@@ -820,8 +823,9 @@ def run_pkv(args):
     # ---- end to end through the public API with host buffers -------------------------
     # Every step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs) from pinned
     # host memory and reads its output back.  "serial": one step at a time, synchronised.
-    # "pipelined": two input buffer sets; the copies of step i+1 run on a copy stream while
-    # step i computes, and the host waits for each step's output one step behind.
+    # "pipelined": E2E_BUFS input/output buffer sets; the copies of step i+1 run on a copy
+    # stream while step i computes, the output copies on a third stream, and the host waits
+    # for each step's output E2E_BUFS - 1 steps behind (room for host-side jitter).
     host_in = {"q": q, "kn": kn, "vn": vn, "slots": slots, "bt": bt, "lens": lens,
                "pairs": pairs_d}
     pin = {k: v.cpu().pin_memory() for k, v in host_in.items()}
@@ -831,11 +835,12 @@ def run_pkv(args):
     torch.cuda.synchronize()
     main = torch.cuda.Stream(device)          # graphs are captured on non-default streams
     copy_stream = torch.cuda.Stream(device)
-    bufs = [host_in, {k: v.clone() for k, v in host_in.items()}]
-    outs = [out, torch.empty_like(out)]
-    outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d_done = [torch.cuda.Event() for _ in range(2)]
-    used = [torch.cuda.Event() for _ in range(2)]
+    nbuf = E2E_BUFS
+    bufs = [host_in] + [{k: v.clone() for k, v in host_in.items()} for _ in range(nbuf - 1)]
+    outs = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
+    outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(nbuf)]
+    h2d_done = [torch.cuda.Event() for _ in range(nbuf)]
+    used = [torch.cuda.Event() for _ in range(nbuf)]
 
     def run_kernels(b):
         d = bufs[b]
@@ -860,32 +865,32 @@ def run_pkv(args):
     # Each half of a step (the input copies; the kernels plus the output copy) is captured
     # once per buffer set as a CUDA graph, so a step costs the host two graph launches.
     g_copy, g_comp = [], []
-    for b in range(2):
+    for b in range(nbuf):
         with torch.cuda.stream(main):
             run_kernels(b)                 # warm the library paths outside capture
         main.synchronize()
-        gc = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gc, stream=copy_stream):
+        gcp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gcp, stream=copy_stream):
             for k, t in bufs[b].items():
                 if k != "pairs" or npairs:
                     t.copy_(pin[k], non_blocking=True)
         gk = torch.cuda.CUDAGraph()
         with torch.cuda.graph(gk, stream=main):
             run_kernels(b)
-        g_copy.append(gc)
+        g_copy.append(gcp)
         g_comp.append(gk)
     torch.cuda.synchronize()
     d2h_stream = torch.cuda.Stream(device)
-    k_done = [torch.cuda.Event() for _ in range(2)]
+    k_done = [torch.cuda.Event() for _ in range(nbuf)]
 
     def e2e_pipelined(n):
         with torch.cuda.stream(copy_stream):
             g_copy[0].replay()
         h2d_done[0].record(copy_stream)
         for i in range(n):
-            b = i & 1
+            b = i % nbuf
             if i + 1 < n:          # stage the next step's inputs behind its buffer's last use
-                nb = (i + 1) & 1
+                nb = (i + 1) % nbuf
                 copy_stream.wait_event(used[nb])
                 with torch.cuda.stream(copy_stream):
                     g_copy[nb].replay()
@@ -898,19 +903,20 @@ def run_pkv(args):
             with torch.cuda.stream(d2h_stream):
                 outs_h[b].copy_(outs[b], non_blocking=True)
             used[b].record(d2h_stream)
-            if i >= 1:
-                used[(i - 1) & 1].synchronize()   # host has step i-1's output
+            if i >= nbuf - 1:      # the host has step i-(nbuf-1)'s output
+                used[(i - nbuf + 1) % nbuf].synchronize()
         d2h_stream.synchronize()
         main.synchronize()
 
     # pipelined e2e: at least 1000 steps (about 0.13 s on the headline batch), so that the
-    # two-deep pipeline's fill and drain and the first replays of the freshly captured graphs
+    # pipeline's fill and drain and the first replays of the freshly captured graphs
     # do not dominate a short run
     Ke = max(1000, K)
     Ks = max(1, min(K, 1000))     # serial mode: at most 1000 synchronised steps
     for _ in range(max(3, args.warmup // 4)):
         e2e_serial_step()
-    e2e_pipelined(4)
+    e2e_pipelined(4 * nbuf)
+    gc.disable()                  # no collector pauses inside the host-driven loops
     barrier(dist, device)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -930,6 +936,7 @@ def run_pkv(args):
     e1.record(main)                # e2e_pipelined returned after the last output landed
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
+    gc.enable()
     e2e_ms = max_over_ranks(dist, e0.elapsed_time(e1) / Ke, device)
     barrier(dist, device)
     faults = B.device_faults(clear=True)
@@ -1014,7 +1021,9 @@ def run_pkv(args):
                     "steps": Ke, "mode": "pipelined: input copies of step i+1 and the output "
                                           "copy of step i-1 overlap step i's kernels "
                                           "(three streams, kernels and input copies "
-                                          "replayed as CUDA graphs)",
+                                          "replayed as CUDA graphs; %d buffer sets, the "
+                                          "host reads each output %d steps behind)"
+                                          % (E2E_BUFS, E2E_BUFS - 1),
                     "serial_value": round(world * nbytes["kv"] / (e2e_serial_ms * 1e-3) / 1e9,
                                           2),
                     "serial_ms_per_step": round(e2e_serial_ms, 5),
