@@ -144,10 +144,9 @@ struct DecodeFp8Cfg {
     }
 };
 
-// Resident warps per SM the register budget is sized for: 18 gives 2-warp CTAs 112
-// registers a thread (9 CTAs per SM) without spills, measured +0.4 % (gqa) and +1.9 % (long)
-// over 16; 20 (96 registers) is slower, 24 spills.  4-warp CTAs (one query head per kv head)
-// stay at 4 per SM.
+// Resident warps per SM the register cap is sized for.  With 18, the 2-warp CTAs compile to
+// 96 registers (10 CTAs per SM) and the 4-warp CTAs (one query head per kv head) to 124 (4
+// per SM); 16 and 20 measured 1-4 % slower on the grouped-head batches, 24 spills.
 #ifndef PKV_FP8_WARPS_PER_SM
 #define PKV_FP8_WARPS_PER_SM 18
 #endif
