@@ -102,6 +102,22 @@ def test_split_partitions_and_lse_reduce(pt, dtype):
     assert err <= TOL[dtype], (pt, err)
 
 
+@pytest.mark.parametrize("longest", [2048, 2049, 16384, 16400])
+def test_lse_reduce_one_warp_and_eight_warp_rows(longest):
+    """The reduce takes one warp per row while no row has more than 8 partitions and 8 warps
+    per row beyond that (each warp loading batches of 8 partitions, rescaling its sums when a
+    later batch holds a larger max).  256-token partitions: the longest sequence gives 8
+    partitions (one warp), 9 (eight warps, one partition for most), 64 (eight warps, one full
+    batch each) or 65 (a second batch for warp 0).  Every row count from 1 up is present;
+    fp32 holds the merge to 1e-5."""
+    lens = [1, 16, 255, 256, 257, 511, 513, 1023, 1025, 1500, 2047, longest]
+    wl = small_wl(lens, 4, 2, 64, "f32", seed=longest, partition_tokens=256)
+    vals = W.make_values(wl, "cpu")
+    got, ref = run_step(wl, vals)
+    err = np.max(np.abs(got - ref))
+    assert err <= TOL["f32"], (longest, err)
+
+
 def test_split_and_unsplit_agree_closely():
     wl = small_wl([3000, 1800, 4096], 4, 4, 128, "f32", seed=5)
     vals = W.make_values(wl, "cpu")
