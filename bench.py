@@ -550,6 +550,39 @@ def swap_probe(torch, B, wl, kp, vp, device, reps=5):
     return res
 
 
+def time_block_manager(B, wl, steps=200):
+    """Host cost of one decode step's block-manager work for this batch: append one slot to
+    every sequence (on-demand block allocation, copy-on-write decisions) and export the
+    padded block tables, through the C ABI from Python (the binding's marshalling included).
+    The sequences start one token short of the workload's lengths and grow by one a step."""
+    import time
+    S = wl.num_seqs
+    lens = [int(x) for x in wl.context_lens]
+    grow = (steps + wl.block_size - 1) // wl.block_size + 1
+    nb = int(sum((L + wl.block_size - 1) // wl.block_size + grow for L in lens))
+    bm = B.BlockManager(nb, block_size=wl.block_size)
+    try:
+        for i, L in enumerate(lens):
+            bm.add_seq(i, L - 1)
+        seqs = list(range(S))
+        maxb = max((L + steps + wl.block_size - 1) // wl.block_size for L in lens)
+        t_app = t_tab = 0.0
+        for _ in range(steps):
+            t0 = time.perf_counter()
+            bm.append_slots(seqs)
+            t1 = time.perf_counter()
+            bm.block_tables(seqs, maxb)
+            t2 = time.perf_counter()
+            t_app += t1 - t0
+            t_tab += t2 - t1
+    finally:
+        bm.close()
+    return {"append_slots_us": round(t_app / steps * 1e6, 2),
+            "block_tables_us": round(t_tab / steps * 1e6, 2), "seqs": S, "steps": steps,
+            "what": "host C++ block manager per decode step through the Python binding: "
+                    "one slot for every sequence, then the padded [S, max_blocks] tables"}
+
+
 def time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ksc, vsc,
                      nbytes, calls=20, reps=10):
     """kv_write (or kv_write_fp8) of the step's new tokens and kv_copy_blocks, each timed
@@ -952,6 +985,7 @@ def run_pkv(args):
 
     result = None
     if rank == 0:
+        bm_host = time_block_manager(B, wl)
         peak, peak_kind = hbm_peak()
         step_ms = ms / K
         kv_gbs = world * nbytes["kv"] / (step_ms * 1e-3) / 1e9
@@ -1031,6 +1065,7 @@ def run_pkv(args):
                           "working set larger than L2"},
             "gpu_launches": K * launches_per_step,
             "write_and_copy_kernels": aux,
+            "block_manager_host": bm_host,
             "kv_utilisation": kv_utilisation(wl),
             "swap": swap,
             "clocks": sampler.summary(),

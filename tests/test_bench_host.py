@@ -155,3 +155,14 @@ def test_both_arms_describe_the_step_with_one_config():
     c2 = bench.step_config(args, wl2, len(pairs2), 512, nb,
                            bench.uses_l2_flush(args, wl2, nb, False), False)
     assert c1 == c2 and c1["cow_pairs_per_step"] == 112
+
+
+def test_block_manager_host_timing_leaves_no_sequence_behind():
+    """The bench's host timing of one step's block-manager work: it must run on the host
+    alone (no GPU), append exactly one slot per sequence per step, and report both parts."""
+    from paged_kv_cache_392_b200 import binding as B
+    from paged_kv_cache_392_b200 import workloads as W
+    wl = W.make_workload("bm", [5, 17, 33, 48, 1], 2, 2, 64, "f32", 3)
+    r = bench.time_block_manager(B, wl, steps=40)
+    assert r["seqs"] == 5 and r["steps"] == 40
+    assert r["append_slots_us"] > 0 and r["block_tables_us"] > 0
