@@ -155,7 +155,7 @@ constexpr int kFp8WarpsPerSm = PKV_FP8_WARPS_PER_SM;
 // T: the q / out type (__half or __nv_bfloat16); the pools are E4M3 bytes.  G query heads
 // per kv head, W warps per CTA, NSW ring stages per warp, BSH log2 of the tokens per physical
 // block (4 or 5: a compile-time constant here, so that the block addressing of the 16-token
-// blocks costs this instruction-bound kernel nothing; it must equal DecodeParams::bshift).
+// blocks costs nothing; it must equal DecodeParams::bshift).
 template <typename T, int G, int W, int NSW, int BSH>
 __global__ void __launch_bounds__(W * 32, kFp8WarpsPerSm / W)
 paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
