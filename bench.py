@@ -9,7 +9,7 @@ the two calls.
     python bench.py [--gpus N] [--steps K] [--warmup W]
                     [--workload opt13b|gqa|long|fork|beam|prefix|tiny] [--kv-fp8]
                     [--impl pkv|reference] [--no-cpu-baseline] [--separate-write]
-                    [--l2-flush] [--swap-probe] [--read-probe] [--contiguous]
+                    [--l2-flush] [--swap-probe] [--no-read-probe] [--contiguous]
                     [--layout paged|contiguous] [--decode-only] [--lib-defines '-D...']
 
 N > 1 runs under torchrun, one process per GPU; every rank decodes its own replica of the
@@ -73,8 +73,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="pkv", choices=["pkv", "reference"])
     ap.add_argument("--partition-tokens", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--read-probe", action="store_true",
-                    help="also measure a read-only streaming ceiling (torch.sum, 2 GiB)")
+    ap.add_argument("--no-read-probe", action="store_true",
+                    help="skip the read-bandwidth probe (the library's streaming copy of a "
+                         "4 GiB buffer in the decode's chunk size) reported beside the peak")
     ap.add_argument("--kv-fp8", action="store_true",
                     help="FP8 (E4M3) KV cache: kv_write_fp8 + paged_attn_decode_fp8 "
                          "(opt13b, gqa, long)")
@@ -641,21 +642,30 @@ def time_aux_kernels(torch, B, wl, pairs, kp, vp, kn, vn, slots, device, fp8, ks
     return res
 
 
-def read_probe_gbs(torch, device, gib=2, reps=5):
-    """Best-of-reps read bandwidth of a plain streaming reduction (torch.sum over a 2 GiB
-    bf16 buffer): a read-only ceiling to set beside the copy-based peak."""
-    x = torch.ones(gib << 29, dtype=torch.bfloat16, device=device)
-    best = 0.0
-    for _ in range(reps + 1):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        x.sum(dtype=torch.float32)
-        b.record()
-        torch.cuda.synchronize()
-        best = max(best, x.numel() * 2 / (a.elapsed_time(b) * 1e-3) / 1e9)
+def read_probe_gbs(torch, B, device, chunk, gib=4, reps=3, per_sm=(2, 4, 6, 8, 0)):
+    """The library's streaming probe (pkv_read_probe: pseudo-randomly permuted chunk-sized
+    bulk copies of a gib-GiB buffer into shared memory, nothing else), best over reps and over
+    a few concurrencies (CTAs per SM; 0 = as many as fit): the read ceiling for copies of the
+    decode's size, set beside the copy-based peak.  Returns (GB/s, CTAs per SM of the best)."""
+    x = torch.empty(gib << 30, dtype=torch.uint8, device=device)
+    x.fill_(1)
+    best, best_per = 0.0, None
+    for per in per_sm:
+        for _ in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            n = B.read_probe(x, chunk, per)
+            b.record()
+            torch.cuda.synchronize()
+            gbs = n / (a.elapsed_time(b) * 1e-3) / 1e9
+            if gbs > best:
+                best, best_per = gbs, per
+    faults = B.device_faults(clear=True)
     del x
     torch.cuda.empty_cache()
-    return round(best, 1)
+    if faults:
+        raise RuntimeError("device faults in the read probe: %s" % faults)
+    return round(best, 1), best_per
 
 
 # ---- the CUDA path --------------------------------------------------------------------------
@@ -998,7 +1008,11 @@ def run_pkv(args):
         achieved = decode_call_bytes / (call_ms * 1e-3) / 1e9
         traffic = (None if args.separate_write or decode_only
                    else profile_traffic(args.workload, fp8))
-        probe = read_probe_gbs(torch, device) if args.read_probe else None
+        # one 16-token K (or V) copy of the decode
+        probe_chunk = 16 * wl.head_dim * (1 if fp8 else 4 if wl.dtype == "f32" else 2)
+        probe, probe_per = ((None, None) if args.no_read_probe
+                            else read_probe_gbs(torch, B, device,
+                                                max(2048, min(16384, probe_chunk))))
         swap = swap_probe(torch, B, wl, kp, vp, device) if args.swap_probe and not fp8 else None
         result = {
             "metric": METRIC,
@@ -1038,6 +1052,9 @@ def run_pkv(args):
                 "frac": round(achieved / peak, 4),
                 "frac_of_8TBs_spec": round(achieved / 8000.0, 4),
                 "read_probe_gbs": probe,
+                "read_probe_chunk_bytes": (None if probe is None
+                                           else max(2048, min(16384, probe_chunk))),
+                "read_probe_ctas_per_sm": probe_per,
                 "frac_of_read_probe": round(achieved / probe, 4) if probe else None,
                 "traffic": traffic,
                 "algorithmic_bytes": decode_call_bytes,

@@ -405,6 +405,25 @@ pkv_status pkv_bm_swap_in(pkv_bm *bm, int64_t seq, int32_t *pairs_out, int32_t c
 pkv_status pkv_bm_is_swapped(const pkv_bm *bm, int64_t seq, int32_t *swapped);
 int32_t pkv_bm_num_host_free(const pkv_bm *bm);
 
+/* ---- measurement aid -------------------------------------------------------------------- */
+/*
+ * Read-bandwidth probe (the pages have no counterpart: it gives the roofline a read-only
+ * denominator).  Streams chunk_bytes-sized chunks of the device buffer buf into shared
+ * memory with 1-D bulk copies, in a fixed scattered order (a bijective hash of the chunk
+ * index), and discards them; n is the largest power of two with n * chunk_bytes <= bytes.  Every chunk
+ * is read once; nothing is written.  Time it with events on the stream.
+ *   buf: device pointer, 16-byte aligned, owned by the caller;
+ *   chunk_bytes: 2048, 4096, 8192 or 16384;
+ *   ctas_per_sm: CTAs of 2 warps (4 copies in flight each) launched per SM; 0 = as many as
+ *     fit; more than fit run in turns;
+ *   bytes_read: host out (may be NULL) = n * chunk_bytes.
+ * Errors: PKV_ERR_INVALID for a null or unaligned buf, an unsupported chunk, fewer than one
+ * chunk or more than 2^31 chunks, a negative ctas_per_sm; PKV_ERR_CUDA for a failed launch.  A copy wait that runs
+ * out sets PKV_FAULT_TIMEOUT in the device fault word.
+ */
+pkv_status pkv_read_probe(const void *buf, size_t bytes, int32_t chunk_bytes,
+                          int32_t ctas_per_sm, size_t *bytes_read, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

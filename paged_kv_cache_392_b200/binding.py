@@ -36,7 +36,7 @@ EXPORTS = [
     "kv_swap_out", "kv_swap_in", "pkv_bm_set_host_pool", "pkv_bm_swap_out", "pkv_bm_swap_in",
     "pkv_bm_is_swapped", "pkv_bm_num_host_free", "kv_write_fp8", "paged_attn_decode_fp8",
     "kv_write_and_decode", "kv_write_fp8_and_decode", "pkv_fp8_partition_tokens",
-    "attn_decode_contiguous",
+    "attn_decode_contiguous", "pkv_read_probe",
 ]
 
 
@@ -111,6 +111,7 @@ def lib():
                                    vp], i32),
         "kv_write_fp8_and_decode": ([dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float,
                                      vp, vp, sz, vp], i32),
+        "pkv_read_probe": ([vp, sz, i32, i32, P(sz), vp], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -321,6 +322,19 @@ def paged_attn_decode_no_alloc(q, k_pool, v_pool, block_tables, context_lens, sc
         ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(block_tables),
         _ptr(context_lens), float(scale), _ptr(out), _stream(stream, q.device)))
     return out
+
+
+def read_probe(buf, chunk_bytes=8192, ctas_per_sm=0, stream=None):
+    """Stream the device buffer ``buf`` (any dtype, contiguous) through shared memory in
+    permuted ``chunk_bytes`` copies and discard it; returns the bytes read (the largest
+    power-of-two number of chunks that fits).  A read-bandwidth denominator for the roofline.
+    ``ctas_per_sm`` sets the concurrency (0: as many CTAs as fit)."""
+    if not (isinstance(buf, torch.Tensor) and buf.is_cuda and buf.is_contiguous()):
+        raise ValueError("buf must be a contiguous CUDA tensor")
+    n = ctypes.c_size_t()
+    _check(lib().pkv_read_probe(_ptr(buf), buf.numel() * buf.element_size(), int(chunk_bytes),
+                                int(ctas_per_sm), ctypes.byref(n), _stream(stream, buf.device)))
+    return n.value
 
 
 def kv_write(k_new, v_new, slot_mapping, k_pool, v_pool, stream=None):

@@ -14,6 +14,7 @@
 #include "attn_decode_fp8.cuh"
 #include "attn_decode_tc.cuh"
 #include "kv_ops.cuh"
+#include "read_probe.cuh"
 #include "pkv_internal.h"
 
 namespace {
@@ -943,3 +944,45 @@ pkv_status pkv_device_faults(uint32_t *faults, int clear, void *stream) {
 }
 
 }  // extern "C"
+
+// ---- read-bandwidth probe -------------------------------------------------------------------
+extern "C" pkv_status pkv_read_probe(const void *buf, size_t bytes, int32_t chunk_bytes,
+                                     int32_t ctas_per_sm, size_t *bytes_read, void *stream) {
+    const char *fn = "pkv_read_probe";
+    if (!buf || (reinterpret_cast<uintptr_t>(buf) & 15u))
+        return fail(PKV_ERR_INVALID, "%s: buf null or not 16-byte aligned", fn);
+    if (chunk_bytes != 2048 && chunk_bytes != 4096 && chunk_bytes != 8192 &&
+        chunk_bytes != 16384)
+        return fail(PKV_ERR_INVALID, "%s: chunk_bytes %d (2048, 4096, 8192 or 16384)", fn,
+                    chunk_bytes);
+    const uint64_t chunks = bytes / (uint64_t)chunk_bytes;
+    if (chunks < 1 || chunks > (1ull << 31))
+        return fail(PKV_ERR_INVALID, "%s: %llu chunks (1 .. 2^31)", fn,
+                    (unsigned long long)chunks);
+    uint64_t n = 1;
+    while (n * 2 <= chunks) n *= 2;
+    const int smem = pkv::kProbeWarps * pkv::kProbeStages * chunk_bytes +
+                     pkv::kProbeWarps * pkv::kProbeStages * 8;
+    // the shared-memory limit is set once per device, for the largest chunk
+    const int smem_max = pkv::kProbeWarps * pkv::kProbeStages * 16384 +
+                         pkv::kProbeWarps * pkv::kProbeStages * 8;
+    static std::atomic<bool> done[kMaxDevices];
+    pkv_status st = ensure_smem(pkv::read_probe_kernel, smem_max, done, fn);
+    if (st) return st;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, pkv::read_probe_kernel, pkv::kProbeWarps * 32, smem);
+    if (e != cudaSuccess) return cuda_check(e, fn, "occupancy");
+    const int sms = device_sm_count();
+    if (per_sm < 1 || sms < 1) return fail(PKV_ERR_CUDA, "%s: no resident CTA fits", fn);
+    if (ctas_per_sm < 0) return fail(PKV_ERR_INVALID, "%s: ctas_per_sm %d", fn, ctas_per_sm);
+    if (ctas_per_sm > 0) per_sm = ctas_per_sm;   // more than fit simply run in turns
+    const uint32_t grid = (uint32_t)sms * (uint32_t)per_sm;
+    pkv::read_probe_kernel<<<grid, pkv::kProbeWarps * 32, smem,
+                             static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const char *>(buf), (uint32_t)n, (uint32_t)chunk_bytes);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_check(e, fn, "launch");
+    if (bytes_read) *bytes_read = (size_t)(n * (uint64_t)chunk_bytes);
+    return PKV_OK;
+}

@@ -172,3 +172,16 @@ def test_contiguous_decode_rejects_bad_arguments_before_launch(lib):
     d2 = _desc(max_blocks_per_seq=100, partition_tokens=512)
     assert f(ctypes.byref(d2), a, a, a, a, 0.1, a, None, 0, None) == 1
     assert "workspace" in B.last_error()
+
+
+def test_read_probe_rejects_bad_arguments_before_launch(lib):
+    f = lib.pkv_read_probe
+    n = ctypes.c_size_t(7)
+    a = ctypes.c_void_p(1 << 20)
+    assert f(None, 1 << 20, 8192, 0, ctypes.byref(n), None) == 1
+    assert "aligned" in B.last_error()
+    assert f(ctypes.c_void_p((1 << 20) + 8), 1 << 20, 8192, 0, ctypes.byref(n), None) == 1
+    assert f(a, 1 << 20, 1000, 0, ctypes.byref(n), None) == 1    # unsupported chunk
+    assert "chunk_bytes" in B.last_error()
+    assert f(a, 4096, 8192, 0, ctypes.byref(n), None) == 1       # less than one chunk
+    assert n.value == 7                                           # untouched on failure

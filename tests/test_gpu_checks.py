@@ -151,3 +151,16 @@ def test_kv_swap_out_skips_pairs_sharing_a_destination():
     assert B.device_faults() == [DUP]
     assert torch.equal(hk[0], kp[3].cpu()) and torch.equal(hv[2], vp[3].cpu())
     assert torch.count_nonzero(hk[1]) == 0 and torch.count_nonzero(hv[1]) == 0
+
+
+def test_read_probe_streams_a_power_of_two_of_chunks_and_faults_nothing():
+    """The bandwidth probe reads the largest power-of-two number of chunks that fits and
+    leaves the device fault word clean; the buffer is only read."""
+    buf = torch.arange(5 << 20, dtype=torch.int32, device="cuda")      # 20 MiB
+    ref = buf.clone()
+    for chunk in (2048, 4096, 8192, 16384):
+        n = B.read_probe(buf, chunk)
+        assert n == (16 << 20)                    # 2^k chunks: 16 MiB of the 20 MiB
+    torch.cuda.synchronize()
+    assert B.device_faults(clear=True) == []
+    assert torch.equal(buf, ref)
