@@ -405,15 +405,25 @@ def _code_only(text):
     return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
 
 
+def _launcher_fp8_section(text):
+    """The FP8 part of the launcher file: from its section banner to the next banner."""
+    a = text.index("// ---- FP8 (E4M3) KV cache")
+    j = text.find("\n// ---- ", a + 1)
+    return text[a:j + 1] if j >= 0 else text[a:]
+
+
 def kernel_source_sha(fp8=False):
     """Hash of the decode kernels' code (kernels and their launch shape; comments left out);
-    the FP8 kernel's launch constants live in the launcher, so its hash covers that file
-    too."""
+    the FP8 kernel's launch constants live in the launcher's FP8 section, so its hash covers
+    that section too."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_392_b200", "csrc")
     for name in (DECODE_FP8_SOURCES if fp8 else DECODE_SOURCES):
         with open(os.path.join(csrc, name)) as f:
-            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
+            text = f.read()
+        if name == "pkv_cuda.cu":
+            text = _launcher_fp8_section(text)
+        h.update(name.encode() + b"\0" + _code_only(text).encode())
     return h.hexdigest()[:16]
 
 
