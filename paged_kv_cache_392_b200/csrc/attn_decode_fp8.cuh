@@ -176,6 +176,36 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     const int rest = bid / p.pmax;
     const int hk = rest % p.Hkv;
     const int s = rest / p.Hkv;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2;
+    const int tq = lane & 3;
+    const int j0 = part * p.part_blocks;
+    const int32_t *btab = p.block_tables + (size_t)s * p.maxB;
+    const int j1 = j0 + warp;  // this warp's first sub-block
+
+    // Loads that need no context length start with it, so that a unit's start costs one
+    // round trip less: this lane's query values (four 16-bit values a load) and the warp's
+    // first 32 table entries (entries past the sequence's end lie inside its table row and
+    // are never used).
+    constexpr int K32 = D / 32;
+    const bool hv = g < G;
+    uint2 qraw[K32][2];
+    {
+        const T *qrow =
+            static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
+#pragma unroll
+        for (int j = 0; j < K32; ++j)
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+                qraw[j][b] = hv ? *reinterpret_cast<const uint2 *>(qrow + 32 * j + 16 * b + 4 * tq)
+                                : make_uint2(0u, 0u);
+    }
+    int32_t tab;
+    {
+        const int e = sub_to_entry(j1 + W * lane, BSH);
+        tab = e < p.maxB ? btab[e] : 0;
+    }
 
     const int L = p.context_lens[s];
     if (L < 1 || L > (p.maxB << BSH)) {
@@ -185,13 +215,7 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     const int nblk = (L + kBlock - 1) / kBlock;
     const int nparts = (nblk + p.part_blocks - 1) / p.part_blocks;
     if (part >= nparts) return;
-    const int j0 = part * p.part_blocks;
     const int nb = min(nblk, j0 + p.part_blocks) - j0;
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g = lane >> 2;
-    const int tq = lane & 3;
     const int nbw = nb > warp ? (nb - warp + W - 1) / W : 0;
 
     unsigned char *ring = smem + warp * NSW * C::STAGE;
@@ -209,12 +233,9 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     if (p.slot_mapping != nullptr && part == nparts - 1 && warp == (nb - 1) % W)
         write_newest_token_fp8<T, BSH>(fp, s, hk, L, lane);
 
-    const int32_t *btab = p.block_tables + (size_t)s * p.maxB;
-    const int j1 = j0 + warp;  // this warp's first sub-block
     const char *vbase = static_cast<const char *>(p.v_pool);
     const uint64_t policy = l2_evict_first_policy();
     int tab_chunk = 0;
-    int32_t tab = lane < nbw ? btab[sub_to_entry(j1 + W * lane, BSH)] : 0;
 
     auto issue = [&](int i) {
         if ((i >> 5) != tab_chunk) {
@@ -257,30 +278,28 @@ paged_attn_decode_fp8_kernel(const __grid_constant__ CUtensorMap tmk,
     // qh[j][b][0] (the first two) and qh[j][b][1].  A bf16 q row is scaled by a power of two
     // qf (its largest |q| lands in [2^14, 2^15)), so that f16 holds every value exactly
     // except those 2^-28 below the row's largest; an f16 q is used as is.
-    constexpr int K32 = D / 32;
     uint32_t qh[K32][2][2];
     float qf_mine = 1.f;
     {
-        const bool hv = g < G;
-        const T *qrow = static_cast<const T *>(p.q) + ((size_t)s * p.Hq + hk * G + (hv ? g : 0)) * D;
         float qv[K32][2][4];
         float amax = 0.f;
 #pragma unroll
         for (int j = 0; j < K32; ++j)
 #pragma unroll
-            for (int b = 0; b < 2; ++b)
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t w[2] = {qraw[j][b].x, qraw[j][b].y};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float v = 0.f;
-                    if (hv) {
-                        if constexpr (std::is_same<T, __half>::value)
-                            v = __half2float(qrow[32 * j + 16 * b + 4 * tq + e]);
-                        else
-                            v = __bfloat162float(qrow[32 * j + 16 * b + 4 * tq + e]);
-                    }
+                    const uint16_t bits = static_cast<uint16_t>(w[e >> 1] >> (16 * (e & 1)));
+                    float v;
+                    if constexpr (std::is_same<T, __half>::value)
+                        v = __half2float(__ushort_as_half(bits));
+                    else
+                        v = __bfloat162float(__ushort_as_bfloat16(bits));
                     qv[j][b][e] = v;
                     amax = fmaxf(amax, fabsf(v));
                 }
+            }
         if constexpr (!std::is_same<T, __half>::value) {
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
