@@ -1016,8 +1016,9 @@ def run_pkv(args):
         bracketed = decode_call_bytes / (decode_ms * 1e-3) / 1e9
         call_ms = step_ms if only_call else decode_ms
         achieved = decode_call_bytes / (call_ms * 1e-3) / 1e9
-        traffic = (None if args.separate_write or decode_only
-                   else profile_traffic(args.workload, fp8))
+        # the committed summaries were taken on 16-token blocks in the paged layout
+        traffic = (None if args.separate_write or decode_only or contig
+                   or wl.block_size != 16 else profile_traffic(args.workload, fp8))
         # one 16-token K (or V) copy of the decode
         probe_chunk = 16 * wl.head_dim * (1 if fp8 else 4 if wl.dtype == "f32" else 2)
         probe, probe_per = ((None, None) if args.no_read_probe
