@@ -877,8 +877,8 @@ def run_pkv(args):
     # Every step copies its inputs (q, new K/V, slots, tables, lengths, copy pairs) from pinned
     # host memory and reads its output back.  "serial": one step at a time, synchronised.
     # "pipelined": E2E_BUFS input/output buffer sets; the copies of step i+1 run on a copy
-    # stream while step i computes, the output copies on a third stream, and the host waits
-    # for each step's output E2E_BUFS - 1 steps behind (room for host-side jitter).
+    # stream while step i computes and step i-1's output copies on a third stream (all three
+    # in one graph a step), and the host stays at most E2E_BUFS - 1 steps ahead.
     host_in = {"q": q, "kn": kn, "vn": vn, "slots": slots, "bt": bt, "lens": lens,
                "pairs": pairs_d}
     pin = {k: v.cpu().pin_memory() for k, v in host_in.items()}
@@ -892,8 +892,6 @@ def run_pkv(args):
     bufs = [host_in] + [{k: v.clone() for k, v in host_in.items()} for _ in range(nbuf - 1)]
     outs = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
     outs_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(nbuf)]
-    h2d_done = [torch.cuda.Event() for _ in range(nbuf)]
-    used = [torch.cuda.Event() for _ in range(nbuf)]
 
     def run_kernels(b):
         d = bufs[b]
@@ -915,50 +913,53 @@ def run_pkv(args):
             outs_h[0].copy_(outs[0], non_blocking=True)
         main.synchronize()
 
-    # Each half of a step (the input copies; the kernels plus the output copy) is captured
-    # once per buffer set as a CUDA graph, so a step costs the host two graph launches.
-    g_copy, g_comp = [], []
+    # One CUDA graph per buffer phase holds a whole pipelined step on three streams: the
+    # kernels of step i (buffer set i mod n) on the compute stream, the input copies of step
+    # i+1 into the next set on a copy stream, and the output copy of step i-1 on a third.
+    # Graph launches on one stream run in order, so buffer reuse needs no other sync, and a
+    # step costs the host one graph launch.
+    d2h_stream = torch.cuda.Stream(device)
     for b in range(nbuf):
         with torch.cuda.stream(main):
             run_kernels(b)                 # warm the library paths outside capture
         main.synchronize()
-        gcp = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gcp, stream=copy_stream):
-            for k, t in bufs[b].items():
-                if k != "pairs" or npairs:
-                    t.copy_(pin[k], non_blocking=True)
-        gk = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gk, stream=main):
+    g_step = []
+    for b in range(nbuf):
+        nxt, prv = (b + 1) % nbuf, (b - 1) % nbuf
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=main):
+            fork = torch.cuda.Event()
+            fork.record(main)
+            copy_stream.wait_event(fork)
+            d2h_stream.wait_event(fork)
+            with torch.cuda.stream(copy_stream):
+                for k, t in bufs[nxt].items():
+                    if k != "pairs" or npairs:
+                        t.copy_(pin[k], non_blocking=True)
+            with torch.cuda.stream(d2h_stream):
+                outs_h[prv].copy_(outs[prv], non_blocking=True)
             run_kernels(b)
-        g_copy.append(gcp)
-        g_comp.append(gk)
+            j1, j2 = torch.cuda.Event(), torch.cuda.Event()
+            j1.record(copy_stream)
+            j2.record(d2h_stream)
+            main.wait_event(j1)
+            main.wait_event(j2)
+        g_step.append(g)
     torch.cuda.synchronize()
-    d2h_stream = torch.cuda.Stream(device)
-    k_done = [torch.cuda.Event() for _ in range(nbuf)]
+    step_done = [torch.cuda.Event() for _ in range(nbuf)]
 
     def e2e_pipelined(n):
-        with torch.cuda.stream(copy_stream):
-            g_copy[0].replay()
-        h2d_done[0].record(copy_stream)
+        h2d_copy(0, main)                  # fill: the first step's inputs
         for i in range(n):
             b = i % nbuf
-            if i + 1 < n:          # stage the next step's inputs behind its buffer's last use
-                nb = (i + 1) % nbuf
-                copy_stream.wait_event(used[nb])
-                with torch.cuda.stream(copy_stream):
-                    g_copy[nb].replay()
-                h2d_done[nb].record(copy_stream)
-            main.wait_event(h2d_done[b])
             with torch.cuda.stream(main):
-                g_comp[b].replay()
-            k_done[b].record(main)
-            d2h_stream.wait_event(k_done[b])      # output copy off the compute stream
-            with torch.cuda.stream(d2h_stream):
-                outs_h[b].copy_(outs[b], non_blocking=True)
-            used[b].record(d2h_stream)
-            if i >= nbuf - 1:      # the host has step i-(nbuf-1)'s output
-                used[(i - nbuf + 1) % nbuf].synchronize()
-        d2h_stream.synchronize()
+                g_step[b].replay()
+            step_done[b].record(main)
+            if i >= nbuf - 1:              # the host is at most nbuf - 1 steps ahead
+                step_done[(i - nbuf + 1) % nbuf].synchronize()
+        last = (n - 1) % nbuf              # drain: the last step's output
+        with torch.cuda.stream(main):
+            outs_h[last].copy_(outs[last], non_blocking=True)
         main.synchronize()
 
     # pipelined e2e: at least 1000 steps (about 0.13 s on the headline batch), so that the
@@ -1082,9 +1083,8 @@ def run_pkv(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": Ke, "mode": "pipelined: input copies of step i+1 and the output "
                                           "copy of step i-1 overlap step i's kernels "
-                                          "(three streams, kernels and input copies "
-                                          "replayed as CUDA graphs; %d buffer sets, the "
-                                          "host reads each output %d steps behind)"
+                                          "(three streams in one CUDA graph a step; %d "
+                                          "buffer sets, the host at most %d steps ahead)"
                                           % (E2E_BUFS, E2E_BUFS - 1),
                     "serial_value": round(world * nbytes["kv"] / (e2e_serial_ms * 1e-3) / 1e9,
                                           2),
